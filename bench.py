@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the ConvRot packed-INT4 quantized linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch: fused rotate+quant (K1)
+of x (8192 x 3840 bf16, G = 64) into packed int4, then the tcgen05 W4A4 GEMM
+with the rowwise-scale epilogue (K2) against packed int4 weights
+(3840 x 3840) -> bf16 y. `value` = 2*M*N*K per step / step time, in TOPS, summed
+over ranks (weak scaling: every rank runs its own replica, no collective on
+the data path) and divided by the slowest rank's time.
+
+Also reported on the same JSON line: per-kernel times and the roofline of the
+dominant kernel (K2, against the int8 tensor peak derived from the measured
+bf16 peak), the end-to-end number through the C ABI with host buffers, the
+W4A8 / AWQ W4A16 decode GEMVs in weight GB/s, SM clocks sampled during the
+timed region, and the CPU oracle timed on a bounded sample (cpu_baseline).
+`--impl reference` times the CPU oracle itself as the reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_linear_rotate_b200 import workloads as WL  # noqa: E402
+
+METRIC = "W4A4 linear TOPS (M=8192) + W4A8/W4A16 GEMV weight GB/s, % of B200 roofline"
+L2_BYTES = 126 * 1024 * 1024
+INT8_PER_BF16 = 2.0      # nominal dense int8 / bf16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "bit_quantized_linear_rotate_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this exact source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self._h = N.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = N.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self._h, N.NVML_CLOCK_SM)
+            self._N = N
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        N = self._N
+        get_r = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            N.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(N.nvmlDeviceGetClockInfo(self._h, N.NVML_CLOCK_SM))
+                r = get_r(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        dist.barrier()
+
+
+# ------------------------------------------------------------ CPU oracle legs
+
+def oracle_linear_sample(w, rows: int):
+    """Times the oracle (as it stands) on the first `rows` rows of the workload."""
+    import oracle as O
+    d = WL.linear_inputs(w)
+    x = d["x"][:rows].float().numpy().astype(np.float64)
+    wp = d["w_packed"].numpy()
+    sw = d["w_scale"].float().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    O.linear_w4a4(x, wp, sw, w.G)
+    dt = time.perf_counter() - t0
+    return dt
+
+
+def cpu_baseline(w, rows: int):
+    dt = oracle_linear_sample(w, rows)
+    ops = 2.0 * rows * w.N * w.K
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {rows} of {w.M} rows of {w.name} (full K, N), one pass, {dt:.2f} s"}
+
+
+# ------------------------------------------------------------------ GPU legs
+
+def time_linear(ck, w, steps: int, warmup: int, world: int, dev):
+    d = WL.linear_inputs(w)
+    per_copy = d["x"].numel() * 2 + d["w_packed"].numel() + w.M * w.N * 2
+    R = max(2, -(-2 * L2_BYTES // per_copy))
+    xs = [d["x"].to(dev) for _ in range(R)]
+    wps = [d["w_packed"].to(dev) for _ in range(R)]
+    sw = d["w_scale"].to(dev)
+    ys = [torch.empty(w.M, w.N, device=dev, dtype=torch.bfloat16) for _ in range(R)]
+    nq = w.M * (w.K // 2)
+    ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
+    qa = ws[:nq].view(w.M, w.K // 2)
+    off = (nq + 255) // 256 * 256
+    sa = ws[off:off + 4 * w.M].view(torch.float32)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        c = i % R
+        if ev is not None:
+            ev[0].record(stream)
+        ck.rotate_quant_rowwise(xs[c], w.G, 4, q_out=qa, scale_out=sa)
+        if ev is not None:
+            ev[1].record(stream)
+        ck.gemm_w4a4(qa, sa, wps[c], sw, out=ys[c])
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(warmup):
+        step(i)
+    ck.device_error_check()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        start.record(stream)
+        for i in range(steps):
+            step(i, evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ck.device_error_check()
+    total_ms = start.elapsed_time(stop)
+    k1 = [e[0].elapsed_time(e[1]) for e in evs]
+    k2 = [e[1].elapsed_time(e[2]) for e in evs]
+    return {"total_ms": total_ms, "k1_ms": statistics.mean(k1), "k2_ms": statistics.mean(k2),
+            "copies": R, "clocks": clk.summary()}
+
+
+def time_linear_e2e(ck, w, steps: int, warmup: int, dev):
+    """ck_linear_w4a4 with host buffers: pinned H2D of x, the linear, D2H of y, every step."""
+    d = WL.linear_inputs(w)
+    x_h = d["x"].pin_memory()
+    y_h = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(d["x"], device=dev)
+    y_d = torch.empty(w.M, w.N, device=dev, dtype=torch.bfloat16)
+    wp, sw = d["w_packed"].to(dev), d["w_scale"].to(dev)
+    ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        x_d.copy_(x_h, non_blocking=True)
+        ck.linear_w4a4(x_d, wp, sw, w.G, workspace=ws, out=y_d)
+        y_h.copy_(y_d, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return {"value": 2.0 * w.M * w.N * w.K / (ms * 1e-3) / 1e12, "unit": "TOPS",
+            "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": y_h.numel() * 2,
+            "ms_per_step": ms}
+
+
+def time_rotating(fn, n_copies: int, iters: int, warmup: int):
+    for i in range(warmup):
+        fn(i % n_copies)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(iters):
+        fn(i % n_copies)
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
+    out = {}
+    w = WL.GEMV_W4A8
+    for M in w.Ms:
+        d = WL.gemv_w4a8_inputs(w, M)
+        R = max(2, -(-2 * L2_BYTES // d["w_packed"].numel()))
+        wps = [d["w_packed"].to(dev) for _ in range(R)]
+        sw = d["w_scale"].to(dev)
+        xq, xs = ck.rotate_quant_rowwise(d["x"].to(dev), 1, 8)      # rowwise int8, no rotation
+        y = torch.empty(M, w.N, device=dev, dtype=torch.bfloat16)
+        ms = time_rotating(lambda c: ck.gemv_w4a8(xq, xs, wps[c], sw, out=y), R, iters, 10)
+        wbytes = w.N * w.K // 2
+        allb = wbytes + 2 * w.N + M * w.K + 4 * M + 2 * M * w.N
+        out[f"w4a8_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
+                             "all_GBps": allb / (ms * 1e-3) / 1e9,
+                             "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R}
+    w = WL.GEMV_AWQ
+    for M in w.Ms:
+        d = WL.gemv_awq_inputs(w, M)
+        per = d["qweight"].numel() + 2 * (d["wscales"].numel() + d["wzeros"].numel())
+        R = max(2, -(-2 * L2_BYTES // per))
+        qws = [d["qweight"].to(dev) for _ in range(R)]
+        wss = [d["wscales"].to(dev) for _ in range(R)]
+        wzs = [d["wzeros"].to(dev) for _ in range(R)]
+        x = d["x"].to(dev)
+        y = torch.empty(M, w.N, device=dev, dtype=torch.bfloat16)
+        ms = time_rotating(lambda c: ck.gemv_awq_w4a16(x, qws[c], wss[c], wzs[c], group_size=w.G, out=y),
+                           R, iters, 10)
+        wbytes = w.N * w.K // 2
+        allb = per + 2 * M * w.K + 2 * M * w.N
+        out[f"awq_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
+                            "all_GBps": allb / (ms * 1e-3) / 1e9,
+                            "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R}
+    return out
+
+
+# --------------------------------------------------------------------- arms
+
+def run_ours(args, world, rank, local):
+    from bit_quantized_linear_rotate_b200 import ck
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WL.LINEAR_M8192
+    peaks, peak_src = load_peaks()
+    t = time_linear(ck, w, args.steps, args.warmup, world, dev)
+    ms_step = max_over_ranks(t["total_ms"], world) / args.steps
+    ops = 2.0 * w.M * w.N * w.K
+    value = ops * world / (ms_step * 1e-3) / 1e12
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    k2_tops = ops / (t["k2_ms"] * 1e-3) / 1e12
+    k1_bytes = w.M * w.K * 2 + w.M * w.K // 2 + 4 * w.M
+    k1_gbs = k1_bytes / (t["k1_ms"] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+        "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "G": w.G,
+                   "step": "rotate_quant(bits=4) + gemm_w4a4 (bf16 out)",
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs rotated over {t['copies']} copies (> 2x L2)"},
+        "roofline": {"bound": "tensor", "achieved": round(k2_tops, 1), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(k2_tops / int8_peak, 4),
+                     "traffic": load_traffic("gemm_w4_kernel"),
+                     "kernel": "gemm_w4_kernel (K2)",
+                     "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_PER_BF16} (int8/bf16 nominal)"},
+        "kernels": {"rotate_quant_us": round(t["k1_ms"] * 1e3, 2), "gemm_w4a4_us": round(t["k2_ms"] * 1e3, 2),
+                    "rotate_quant_GBps": round(k1_gbs, 1),
+                    "rotate_quant_frac_hbm": round(k1_gbs / peaks["hbm_gbs"], 4),
+                    "rotate_quant_traffic": load_traffic("rotate_quant_kernel")},
+        "gpu_launches": 2 * args.steps,
+        "clocks": t["clocks"],
+    }
+    if not args.skip_e2e:
+        line["e2e"] = time_linear_e2e(ck, w, max(3, min(args.steps, 50)), 3, dev)
+    if not args.skip_siblings:
+        line["siblings"] = time_gemvs(ck, dev, peaks["hbm_gbs"])
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = WL.LINEAR_M8192
+    for _ in range(args.warmup):
+        oracle_linear_sample(w, min(args.cpu_rows, 16))
+    times = [oracle_linear_sample(w, args.cpu_rows) for _ in range(args.steps)]
+    dt = sum(times)
+    ops = 2.0 * args.cpu_rows * w.N * w.K * args.steps
+    v = ops / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "G": w.G,
+                       "step": "CPU oracle linear_w4a4 on a bounded row sample"},
+            "cpu_baseline": {"value": v, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"first {args.cpu_rows} of {w.M} rows per step"},
+            "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=512, help="rows of the CPU oracle sample")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-siblings", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 only; other ranks exit without work or collectives
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

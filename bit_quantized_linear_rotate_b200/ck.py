@@ -1,0 +1,217 @@
+"""Python binding of libck.so (include/ck.h): argument marshalling only.
+
+Every function takes CUDA tensors, passes their device pointers, sizes and the
+current CUDA stream to the C entry point of the same name, and raises
+``CKError`` on a non-OK status. All computation happens in the library's CUDA
+kernels; there is no CPU fallback: importing this module without a built
+libck.so raises ImportError.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libck.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m bit_quantized_linear_rotate_b200.build` "
+        "(the ConvRot kernels have no CPU fallback)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+CK_OK, CK_ERR_INVALID_ARG, CK_ERR_UNSUPPORTED, CK_ERR_CUDA, CK_ERR_TIMEOUT = range(5)
+CK_BF16, CK_FP16 = 0, 1
+STATUS_NAMES = {0: "CK_OK", 1: "CK_ERR_INVALID_ARG", 2: "CK_ERR_UNSUPPORTED", 3: "CK_ERR_CUDA",
+                4: "CK_ERR_TIMEOUT"}
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+# name -> argument types (restype is ck_status = int unless listed below)
+SIGNATURES = {
+    "ck_rotate_quant_rowwise": [_p, _int, _i64, _i64, _i64, _int, _int, _p, _p, _p],
+    "ck_gemm_w4a4": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+    "ck_linear_w4a4_workspace_bytes": [_i64, _i64],
+    "ck_linear_w4a4": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
+    "ck_gemv_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+    "ck_gemv_awq_w4a16": [_p, _int, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p],
+    "ck_gemm_w4a4_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
+    "ck_gemm_w4a8_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
+    "ck_device_error_check": [_p],
+    "ck_selftest_bounded_wait": [_i64, _p],
+    "ck_last_error": [],
+    "ck_version": [],
+}
+_RESTYPES = {"ck_linear_w4a4_workspace_bytes": ctypes.c_size_t,
+             "ck_last_error": ctypes.c_char_p, "ck_version": ctypes.c_char_p}
+
+for _name, _args in SIGNATURES.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _RESTYPES.get(_name, ctypes.c_int)
+
+
+class CKError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.ck_last_error().decode()
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != CK_OK:
+        raise CKError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(dt) -> int:
+    if dt == torch.bfloat16:
+        return CK_BF16
+    if dt == torch.float16:
+        return CK_FP16
+    raise TypeError(f"unsupported dtype {dt} (bf16 or fp16)")
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def _rows(x):
+    """(M, K, ldx) of a tensor whose last dim is contiguous; leading dims are flattened."""
+    if x.stride(-1) != 1:
+        raise ValueError("the last dimension must be contiguous")
+    K = x.shape[-1]
+    if x.dim() == 1:
+        return 1, K, K, x
+    x2 = x if x.dim() == 2 else x.reshape(-1, K)
+    return x2.shape[0], K, x2.stride(0), x2
+
+
+def version() -> str:
+    return lib.ck_version().decode()
+
+
+def last_error() -> str:
+    return lib.ck_last_error().decode()
+
+
+def rotate_quant_rowwise(x, group_size: int, bits: int, q_out=None, scale_out=None, stream=None):
+    """Returns (q, scale): q packed int4 (..., K/2) uint8 for bits=4, int8 (..., K) for bits=8."""
+    _cuda(x)
+    M, K, ldx, x2 = _rows(x)
+    lead = tuple(x.shape[:-1])
+    if q_out is None:
+        q_out = torch.empty(lead + ((K // 2,) if bits == 4 else (K,)), device=x.device,
+                            dtype=torch.uint8 if bits == 4 else torch.int8)
+    if scale_out is None:
+        scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
+    _cuda(q_out, scale_out)
+    _check(lib.ck_rotate_quant_rowwise(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
+                                       _ptr(q_out), _ptr(scale_out), _stream(stream)),
+           "ck_rotate_quant_rowwise")
+    return q_out, scale_out
+
+
+def gemm_w4a4(qa_packed, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):
+    _cuda(qa_packed, a_scale, w_packed, w_scale, bias)
+    M, Kh = qa_packed.shape
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=qa_packed.device, dtype=torch.bfloat16)
+    _check(lib.ck_gemm_w4a4(_ptr(qa_packed), _ptr(a_scale), M, 2 * Kh, N, _ptr(w_packed), _ptr(w_scale),
+                            _ptr(bias), _ptr(out), _stream(stream)), "ck_gemm_w4a4")
+    return out
+
+
+def linear_w4a4_workspace_bytes(M: int, K: int) -> int:
+    return int(lib.ck_linear_w4a4_workspace_bytes(M, K))
+
+
+def linear_w4a4(x, w_packed, w_scale, group_size: int, bias=None, workspace=None, out=None,
+                stream=None):
+    """ConvRot W4A4 linear: y (..., N) bf16 from x (..., K) bf16/fp16 and packed (N, K/2) weights."""
+    _cuda(x, w_packed, w_scale, bias)
+    M, K, ldx, x2 = _rows(x)
+    N = w_packed.shape[0]
+    ws_bytes = linear_w4a4_workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=x.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), device=x.device, dtype=torch.bfloat16)
+    _check(lib.ck_linear_w4a4(_ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size, _ptr(w_packed),
+                              _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream)),
+           "ck_linear_w4a4")
+    return out
+
+
+def gemv_w4a8(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
+    _cuda(xq, x_scale, w_packed, w_scale, bias)
+    M, K = xq.shape
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=xq.device, dtype=torch.bfloat16)
+    _check(lib.ck_gemv_w4a8(_ptr(xq), _ptr(x_scale), M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias),
+                            _ptr(out), _stream(stream)), "ck_gemv_w4a8")
+    return out
+
+
+def gemv_awq_w4a16(x, qweight, wscales, wzeros, bias=None, group_size: int = 64, out=None, stream=None):
+    """``ck.gemv_awq_w4a16(x, qdata, wscales, wzeros, bias=, group_size=)``."""
+    _cuda(x, qweight, wscales, wzeros, bias)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=x.device, dtype=x.dtype)
+    _check(lib.ck_gemv_awq_w4a16(_ptr(x), _dtype_code(x.dtype), M, K, N, group_size, _ptr(qweight),
+                                 _ptr(wscales), _ptr(wzeros), _ptr(bias), _ptr(out), _stream(stream)),
+           "ck_gemv_awq_w4a16")
+    return out
+
+
+def gemm_w4a4_i32(qa_packed, w_packed, out=None, stream=None):
+    _cuda(qa_packed, w_packed)
+    M, Kh = qa_packed.shape
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=qa_packed.device, dtype=torch.int32)
+    _check(lib.ck_gemm_w4a4_i32(_ptr(qa_packed), _ptr(w_packed), M, 2 * Kh, N, _ptr(out), _stream(stream)),
+           "ck_gemm_w4a4_i32")
+    return out
+
+
+def gemm_w4a8_i32(qa, w_packed, out=None, stream=None):
+    _cuda(qa, w_packed)
+    M, K = qa.shape
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=qa.device, dtype=torch.int32)
+    _check(lib.ck_gemm_w4a8_i32(_ptr(qa), _ptr(w_packed), M, K, N, _ptr(out), _stream(stream)),
+           "ck_gemm_w4a8_i32")
+    return out
+
+
+def device_error_check(stream=None) -> None:
+    """Synchronises the stream and raises CKError(CK_ERR_TIMEOUT) if a bounded wait gave up."""
+    _check(lib.ck_device_error_check(_stream(stream)), "ck_device_error_check")
+
+
+def selftest_bounded_wait(timeout_ns: int, stream=None) -> None:
+    _check(lib.ck_selftest_bounded_wait(int(timeout_ns), _stream(stream)), "ck_selftest_bounded_wait")

@@ -1,0 +1,352 @@
+// Host side of the C ABI declared in include/ck.h: argument validation, TMA
+// tensor maps, kernel selection and launches. Everything is enqueued on the
+// caller's stream; nothing here allocates, frees or synchronises, except
+// ck_device_error_check (documented as synchronising).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/ck.h"
+#include "ck_common.cuh"
+#include "gemm_w4a4_sm100.cuh"
+#include "gemv_awq.cuh"
+#include "gemv_w4a8.cuh"
+#include "rotate_quant.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ck_status fail(ck_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+ck_status ok() {
+  g_last_error.clear();
+  return CK_OK;
+}
+
+ck_status launch_status(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(CK_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major byte matrix (rows x cols) with row stride `ld` bytes, box = (box_cols x box_rows).
+ck_status make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
+                    uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(CK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return CK_OK;
+}
+
+// ------------------------------------------------------------------ kernels
+
+// One cache per kernel instantiation (the Tag template argument), per device.
+template <typename Tag, typename KernelT>
+ck_status ensure_smem_attr(KernelT kernel, size_t bytes) {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(CK_ERR_CUDA, "cudaGetDevice failed");
+  if (!done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return fail(CK_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    done[dev] = true;
+  }
+  return CK_OK;
+}
+
+template <int VPT, int BITS, typename T>
+void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s, int nt,
+               cudaStream_t st) {
+  const float rnorm = (float)(1.0 / std::sqrt((double)G));
+  ck::rq::rotate_quant_kernel<VPT, BITS, T><<<(unsigned)M, nt, 0, st>>>(
+      reinterpret_cast<const T*>(x), K, ldx, G, rnorm, reinterpret_cast<uint8_t*>(q), s);
+}
+
+template <int BITS, typename T>
+void launch_rq_vpt(int vpt, const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s,
+                   int nt, cudaStream_t st) {
+  switch (vpt) {
+    case 1: launch_rq<1, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
+    case 2: launch_rq<2, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
+    case 4: launch_rq<4, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
+    default: launch_rq<8, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
+  }
+}
+
+ck_status rotate_quant_impl(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int G,
+                            int bits, void* q, float* s, cudaStream_t st) {
+  const int64_t nvec = K / 8;
+  const int target = M >= 1024 ? 128 : 1024;
+  int vpt = 1;
+  while (vpt < 8 && (nvec + vpt - 1) / vpt > target) vpt *= 2;
+  int64_t nt = ((nvec + vpt - 1) / vpt + 31) / 32 * 32;
+  if (nt > ck::rq::max_threads(vpt))
+    return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K=%lld too large (max 32768)", (long long)K);
+  if (xt == CK_BF16) {
+    if (bits == 4) launch_rq_vpt<4, __nv_bfloat16>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
+    else launch_rq_vpt<8, __nv_bfloat16>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
+  } else {
+    if (bits == 4) launch_rq_vpt<4, __half>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
+    else launch_rq_vpt<8, __half>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
+  }
+  return launch_status("rotate_quant");
+}
+
+ck_status check_gemm_shape(const char* who, int64_t M, int64_t K, int64_t N) {
+  if (M <= 0 || K <= 0 || N <= 0) return fail(CK_ERR_INVALID_ARG, "%s: M, K, N must be > 0", who);
+  if (K % 32 != 0) return fail(CK_ERR_UNSUPPORTED, "%s: K=%lld must be a multiple of 32", who, (long long)K);
+  if (M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2 || K > (int64_t)INT32_MAX / 2)
+    return fail(CK_ERR_UNSUPPORTED, "%s: dimension too large", who);
+  if ((M + ck::gemm::BM - 1) / ck::gemm::BM > 65535)
+    return fail(CK_ERR_UNSUPPORTED, "%s: M=%lld too large for one launch", who, (long long)M);
+  return CK_OK;
+}
+
+template <bool A_PACKED, int EPI>
+ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const uint8_t* w,
+                    const float* a_scale, const uint16_t* w_scale, const uint16_t* bias, void* out,
+                    cudaStream_t st) {
+  using namespace ck::gemm;
+  CUtensorMap ta, tb;
+  ck_status r;
+  if (A_PACKED) r = make_tmap(&ta, qa, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, PKB, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else r = make_tmap(&ta, qa, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (r != CK_OK) return r;
+  r = make_tmap(&tb, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, PKB, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (r != CK_OK) return r;
+  auto kern = gemm_w4_kernel<A_PACKED, EPI>;
+  struct Tag {};
+  if ((r = ensure_smem_attr<Tag>(kern, kSmemBytes)) != CK_OK) return r;
+  Params p;
+  p.M = (int)M; p.N = (int)N; p.K = (int)K;
+  p.a_scale = a_scale;
+  p.w_scale = reinterpret_cast<const __nv_bfloat16*>(w_scale);
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  p.out = out;
+  const size_t esz = EPI == EPI_I32 ? 4 : 2;
+  p.out_vec_ok = aligned(out, 16) && ((N * (int64_t)esz) % 16 == 0);
+  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  kern<<<grid, kThreads, kSmemBytes, st>>>(ta, tb, p);
+  return launch_status("gemm_w4");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ck_last_error(void) { return g_last_error.c_str(); }
+
+const char* ck_version(void) { return "ck 0.1 (sm_100a)"; }
+
+ck_status ck_rotate_quant_rowwise(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                  int group_size, int bits, void* q_out, float* scale_out,
+                                  void* stream) {
+  if (M < 0 || K <= 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant: need M >= 0 and K > 0");
+  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "rotate_quant: unknown dtype");
+  if (bits != 4 && bits != 8) return fail(CK_ERR_INVALID_ARG, "rotate_quant: bits must be 4 or 8");
+  if (!is_pow2(group_size) || group_size > 256)
+    return fail(CK_ERR_UNSUPPORTED, "rotate_quant: group_size=%d must be a power of two <= 256", group_size);
+  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant: K %% group_size != 0");
+  if (K % 8 != 0) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K must be a multiple of 8");
+  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "rotate_quant: ldx < K");
+  if (M == 0) return ok();
+  if (x == nullptr || q_out == nullptr || scale_out == nullptr)
+    return fail(CK_ERR_INVALID_ARG, "rotate_quant: null pointer");
+  if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant: x rows must be 16-byte aligned");
+  if (!aligned(q_out, 16) || !aligned(scale_out, 4)) return fail(CK_ERR_INVALID_ARG, "rotate_quant: misaligned output");
+  if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: M too large");
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, q_out, scale_out, S(stream));
+}
+
+ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M, int64_t K,
+                       int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
+                       const uint16_t* bias, uint16_t* y, void* stream) {
+  ck_status r = check_gemm_shape("gemm_w4a4", M, K, N);
+  if (r != CK_OK) return r;
+  if (!qa_packed || !a_scale || !w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4: null pointer");
+  if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4: operands must be 16-byte aligned");
+  if (!aligned(a_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "gemm_w4a4: misaligned scale, bias or output");
+  return gemm_impl<true, ck::gemm::EPI_BF16>(qa_packed, M, K, N, w_packed, a_scale, w_scale, bias, y, S(stream));
+}
+
+size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  const size_t qa = ((size_t)M * (size_t)(K / 2) + 255) / 256 * 256;
+  return qa + (size_t)M * sizeof(float);
+}
+
+ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
+                         int group_size, const uint8_t* w_packed, const uint16_t* w_scale,
+                         const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  ck_status r = check_gemm_shape("linear_w4a4", M, K, N);
+  if (r != CK_OK) return r;
+  if (!workspace || ws_bytes < ck_linear_w4a4_workspace_bytes(M, K))
+    return fail(CK_ERR_INVALID_ARG, "linear_w4a4: workspace smaller than ck_linear_w4a4_workspace_bytes");
+  if (!aligned(workspace, 256)) return fail(CK_ERR_INVALID_ARG, "linear_w4a4: workspace must be 256-byte aligned");
+  if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "linear_w4a4: null pointer");
+  if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "linear_w4a4: weights must be 16-byte aligned");
+  if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "linear_w4a4: misaligned scale, bias or output");
+  uint8_t* qa = reinterpret_cast<uint8_t*>(workspace);
+  float* sa = reinterpret_cast<float*>(qa + ((size_t)M * (size_t)(K / 2) + 255) / 256 * 256);
+  r = ck_rotate_quant_rowwise(x, xt, M, K, ldx, group_size, 4, qa, sa, stream);
+  if (r != CK_OK) return r;
+  return gemm_impl<true, ck::gemm::EPI_BF16>(qa, M, K, N, w_packed, sa, w_scale, bias, y, S(stream));
+}
+
+ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, int64_t M, int64_t K,
+                           int64_t N, int32_t* acc, void* stream) {
+  ck_status r = check_gemm_shape("gemm_w4a4_i32", M, K, N);
+  if (r != CK_OK) return r;
+  if (!qa_packed || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4_i32: null pointer");
+  if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4_i32: operands must be 16-byte aligned");
+  if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4_i32: misaligned output");
+  return gemm_impl<true, ck::gemm::EPI_I32>(qa_packed, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
+}
+
+ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M, int64_t K, int64_t N,
+                           int32_t* acc, void* stream) {
+  ck_status r = check_gemm_shape("gemm_w4a8_i32", M, K, N);
+  if (r != CK_OK) return r;
+  if (!qa || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8_i32: null pointer");
+  if (!aligned(qa, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a8_i32: operands must be 16-byte aligned");
+  if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8_i32: misaligned output");
+  return gemm_impl<false, ck::gemm::EPI_I32>(qa, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
+}
+
+ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
+                       const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
+                       uint16_t* y, void* stream) {
+  if (M <= 0 || K <= 0 || N <= 0) return fail(CK_ERR_INVALID_ARG, "gemv_w4a8: M, K, N must be > 0");
+  if (M > 16) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: M=%lld > 16", (long long)M);
+  if (K % 128 != 0) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: K must be a multiple of 128");
+  if (K > INT32_MAX / 2 || N > INT32_MAX / 2) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: dimension too large");
+  if (!xq || !x_scale || !w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemv_w4a8: null pointer");
+  if (!aligned(xq, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: operands must be 16-byte aligned");
+  if (!aligned(x_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "gemv_w4a8: misaligned scale, bias or output");
+  const unsigned grid = (unsigned)((N + ck::w4a8::kRows - 1) / ck::w4a8::kRows);
+  const auto* sw = reinterpret_cast<const __nv_bfloat16*>(w_scale);
+  const auto* bb = reinterpret_cast<const __nv_bfloat16*>(bias);
+  auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
+  if (M <= 8)
+    ck::w4a8::gemv_w4a8_kernel<1><<<grid, ck::w4a8::kWarps * 32, 0, S(stream)>>>(xq, x_scale, (int)M, (int)K, (int)N, w_packed, sw, bb, yy);
+  else
+    ck::w4a8::gemv_w4a8_kernel<2><<<grid, ck::w4a8::kWarps * 32, 0, S(stream)>>>(xq, x_scale, (int)M, (int)K, (int)N, w_packed, sw, bb, yy);
+  return launch_status("gemv_w4a8");
+}
+
+ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, int64_t N, int group_size,
+                            const uint8_t* qweight, const void* wscales, const void* wzeros,
+                            const void* bias, void* y, void* stream) {
+  if (M <= 0 || K <= 0 || N <= 0) return fail(CK_ERR_INVALID_ARG, "gemv_awq_w4a16: M, K, N must be > 0");
+  if (dt != CK_BF16 && dt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "gemv_awq_w4a16: unknown dtype");
+  if (M > 8) return fail(CK_ERR_UNSUPPORTED, "gemv_awq_w4a16: M=%lld > 8", (long long)M);
+  if (group_size <= 0 || group_size % 64 != 0)
+    return fail(CK_ERR_UNSUPPORTED, "gemv_awq_w4a16: group_size=%d must be a multiple of 64", group_size);
+  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "gemv_awq_w4a16: K %% group_size != 0");
+  if (K > INT32_MAX / 2 || N > INT32_MAX / 2) return fail(CK_ERR_UNSUPPORTED, "gemv_awq_w4a16: dimension too large");
+  if (!x || !qweight || !wscales || !wzeros || !y) return fail(CK_ERR_INVALID_ARG, "gemv_awq_w4a16: null pointer");
+  if (!aligned(x, 16) || !aligned(qweight, 16)) return fail(CK_ERR_UNSUPPORTED, "gemv_awq_w4a16: x and qweight must be 16-byte aligned");
+  if (!aligned(wscales, 2) || !aligned(wzeros, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "gemv_awq_w4a16: misaligned scales, zeros, bias or output");
+  const unsigned grid = (unsigned)((N + ck::awq::kRows - 1) / ck::awq::kRows);
+  if (dt == CK_BF16) {
+    using T = __nv_bfloat16;
+    ck::awq::gemv_awq_kernel<T><<<grid, ck::awq::kWarps * 32, 0, S(stream)>>>(
+        (const T*)x, (int)M, (int)K, (int)N, group_size, qweight, (const T*)wscales, (const T*)wzeros,
+        (const T*)bias, (T*)y);
+  } else {
+    using T = __half;
+    ck::awq::gemv_awq_kernel<T><<<grid, ck::awq::kWarps * 32, 0, S(stream)>>>(
+        (const T*)x, (int)M, (int)K, (int)N, group_size, qweight, (const T*)wscales, (const T*)wzeros,
+        (const T*)bias, (T*)y);
+  }
+  return launch_status("gemv_awq_w4a16");
+}
+
+ck_status ck_device_error_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return fail(CK_ERR_CUDA, "stream error: %s", cudaGetErrorString(e));
+  unsigned int w = 0;
+  e = cudaMemcpyFromSymbol(&w, ck::g_err_word, sizeof(w));
+  if (e != cudaSuccess) return fail(CK_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+  if (w != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(ck::g_err_word, &zero, sizeof(zero));
+    return fail(CK_ERR_TIMEOUT, "a bounded barrier wait gave up (error word 0x%08x, site %u)", w, (w >> 8) & 0xffu);
+  }
+  return ok();
+}
+
+}  // extern "C"
+
+namespace {
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ck::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ck::fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ck::mbar_wait(&bar, 0, &abort_flag, 0x7f, limit_ns);  // nothing arrives
+  __syncthreads();
+}
+}  // namespace
+
+extern "C" ck_status ck_selftest_bounded_wait(int64_t timeout_ns, void* stream) {
+  if (timeout_ns < 1000 || timeout_ns > 5000000000ll)
+    return fail(CK_ERR_INVALID_ARG, "selftest_bounded_wait: timeout_ns outside [1e3, 5e9]");
+  selftest_wait_kernel<<<1, 32, 0, S(stream)>>>((uint64_t)timeout_ns);
+  return launch_status("selftest_bounded_wait");
+}

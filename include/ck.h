@@ -1,0 +1,175 @@
+/*
+ * ck.h -- C ABI of the ConvRot packed-INT4 quantized linear for NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument is a DEVICE pointer owned by the caller, unless the
+ *   argument's comment says otherwise. Nothing is allocated, freed or
+ *   synchronised inside a compute call: arguments are validated on the host,
+ *   then the kernels are enqueued on `stream` and the call returns.
+ * - `stream` is a cudaStream_t passed as an opaque pointer (NULL = the legacy
+ *   default stream).
+ * - Matrices are row-major. A "packed int4" matrix of logical shape (R, C) is
+ *   stored as (R, C/2) bytes: bits 0..3 hold column 2j and bits 4..7 column
+ *   2j+1 (comfy_kitchen/tensor/awq_w4a16.py, module docstring). Each nibble is
+ *   offset binary, u = q + 8, so the signed value is q = u - 8 in [-8, 7];
+ *   int8 and uint8 storage are the same bytes.
+ * - bf16 / fp16 values are passed as 16-bit storage (uint16_t).
+ * - Errors: CK_ERR_INVALID_ARG for null pointers, non-positive sizes,
+ *   inconsistent strides or misaligned pointers; CK_ERR_UNSUPPORTED for shapes
+ *   the kernels decline (the pages' "unsupported-shape decline"); CK_ERR_CUDA
+ *   when a launch fails. Nothing is enqueued when validation fails.
+ *   ck_last_error() returns a thread-local message for the last failure.
+ * - Kernels that wait on shared-memory barriers give up after a bounded time
+ *   and set a device error word instead of hanging; ck_device_error_check()
+ *   reports it.
+ */
+#ifndef CK_H_
+#define CK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CK_OK = 0,
+  CK_ERR_INVALID_ARG = 1,
+  CK_ERR_UNSUPPORTED = 2,
+  CK_ERR_CUDA = 3,
+  CK_ERR_TIMEOUT = 4
+} ck_status;
+
+typedef enum { CK_BF16 = 0, CK_FP16 = 1 } ck_dtype;
+
+/*
+ * Fused group rotation + rowwise symmetric quantization
+ * ("quantize_and_rotate_rowwise" of comfy-kitchen PR #155 "[Feat][Ascend] Add
+ * fused RotateQuant backend", section "What this PR does").
+ *
+ * For every row m of x and every group g of `group_size` consecutive columns:
+ *   y_g = x_g . H_G / sqrt(G)          (Sylvester-ordered Hadamard, fp32)
+ *   s_m = max_k |y[m,k]| / qmax         (qmax = 7 for bits=4, 127 for bits=8;
+ *                                        s_m = 1 for an all-zero row)
+ *   q[m,k] = clamp(round_half_even(y[m,k] / s_m), -qmax, qmax)
+ *
+ * x          : (M, K) bf16 or fp16 (xt), row stride ldx >= K elements,
+ *              16-byte aligned rows (ldx % 8 == 0, x 16-byte aligned).
+ * group_size : 1 (no rotation), 16, 64 or 256; K % group_size == 0, K % 8 == 0.
+ * bits       : 4 -> q_out is (M, K/2) packed int4, u = q + 8, low nibble =
+ *                   even column;
+ *              8 -> q_out is (M, K) int8.
+ * scale_out  : (M) float32, always > 0.
+ * M may be any number of flattened leading dimensions; M == 0 is a no-op.
+ */
+ck_status ck_rotate_quant_rowwise(const void* x, ck_dtype xt, int64_t M, int64_t K,
+                                  int64_t ldx, int group_size, int bits, void* q_out,
+                                  float* scale_out, void* stream);
+
+/*
+ * Integer matmul of packed int4 activations with packed int4 weights, int32
+ * accumulation on the tcgen05 tensor cores, and the rowwise-scale epilogue
+ * (the "EpiRowwise" of comfy-kitchen PR #182, Description):
+ *   acc[m,n] = sum_k qa[m,k] * w[n,k]
+ *   y[m,n]   = bf16_rne( (float(acc) * a_scale[m]) * float(w_scale[n]) (+ bias[n]) )
+ *
+ * qa_packed : (M, K/2) packed int4 (e.g. ck_rotate_quant_rowwise with bits=4).
+ * a_scale   : (M) float32.
+ * w_packed  : (N, K/2) packed int4 weights ("convrot_w4a4", stable-diffusion.cpp
+ *             PR #2276, Summary); 16-byte aligned.
+ * w_scale   : (N) bf16 per-output-row weight scale.
+ * bias      : (N) bf16 or NULL.
+ * y         : (M, N) bf16.
+ * Requires K % 32 == 0 (packed rows are whole 16-byte units for the TMA) and
+ * 16-byte aligned qa_packed / w_packed; otherwise CK_ERR_UNSUPPORTED.
+ */
+ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M, int64_t K,
+                       int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
+                       const uint16_t* bias, uint16_t* y, void* stream);
+
+/* Bytes of device workspace ck_linear_w4a4 needs for M rows of logical width K. */
+size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * The ConvRot W4A4 linear ("public ConvRot W4A4 Linear dispatcher",
+ * comfy-kitchen PR #212; packed formats of stable-diffusion.cpp PR #2276):
+ * ck_rotate_quant_rowwise(bits=4) into `workspace`, then ck_gemm_w4a4.
+ * K is the LOGICAL inner dimension (the packed weight has K/2 bytes per row).
+ * workspace : device buffer of at least ck_linear_w4a4_workspace_bytes(M, K)
+ *             bytes, 256-byte aligned; its contents are scratch.
+ * Other arguments as above.
+ */
+ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N,
+                         int64_t ldx, int group_size, const uint8_t* w_packed,
+                         const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * W4A8 decode GEMV ("W4A8 decode GEMV" of comfy-kitchen PR #182, Description;
+ * "asym_w4a8_int8" of stable-diffusion.cpp PR #2276): int8 activations times
+ * packed int4 weights decoded in registers, int32 accumulation, same epilogue
+ * as ck_gemm_w4a4 with a_scale = x_scale.
+ * xq      : (M, K) int8, 16-byte aligned, 1 <= M <= 16.
+ * x_scale : (M) float32.
+ * Requires K % 128 == 0; otherwise CK_ERR_UNSUPPORTED.
+ */
+ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
+                       const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
+                       uint16_t* y, void* stream);
+
+/*
+ * AWQ W4A16 GEMV ("ck.gemv_awq_w4a16(x, qdata, wscales, wzeros, bias=,
+ * group_size=)", comfy_kitchen/tensor/awq_w4a16.py, _awq_forward):
+ *   W[n,k] = (u[n,k] - 8) * wscales[k/G, n] + wzeros[k/G, n]
+ *   y[m,n] = sum_k x[m,k] W[n,k] (+ bias[n])       (fp32 accumulation)
+ * dt applies to x, wscales, wzeros, bias and y (bf16 or fp16).
+ * x       : (M, K), 1 <= M <= 8, 16-byte aligned.
+ * qweight : (N, K/2) packed uint4, 16-byte aligned.
+ * wscales, wzeros : (K/G, N).
+ * Requires group_size % 64 == 0 and K % group_size == 0; otherwise
+ * CK_ERR_UNSUPPORTED.
+ */
+ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, int64_t N,
+                            int group_size, const uint8_t* qweight, const void* wscales,
+                            const void* wzeros, const void* bias, void* y, void* stream);
+
+/*
+ * Test hooks: raw int32 accumulators acc[m,n] = sum_k qa[m,k] * w[n,k] through
+ * the same tensor-core main loop as ck_gemm_w4a4, so identical quantized
+ * inputs can be compared bit for bit.
+ * ck_gemm_w4a4_i32: qa packed int4 (M, K/2).  ck_gemm_w4a8_i32: qa int8 (M, K).
+ * acc: (M, N) int32. Same shape rules as ck_gemm_w4a4.
+ */
+ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, int64_t M,
+                           int64_t K, int64_t N, int32_t* acc, void* stream);
+ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M, int64_t K,
+                           int64_t N, int32_t* acc, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word set by a
+ * kernel whose bounded barrier wait gave up. Returns CK_ERR_TIMEOUT if it was
+ * set, CK_ERR_CUDA if the stream reported an error, CK_OK otherwise.
+ */
+ck_status ck_device_error_check(void* stream);
+
+/*
+ * Self-test of the bounded wait: launches one block that waits on a
+ * shared-memory barrier nothing will ever complete, gives up after
+ * `timeout_ns` nanoseconds (1e3 .. 5e9), sets the device error word and
+ * returns. ck_device_error_check() must then report CK_ERR_TIMEOUT.
+ */
+ck_status ck_selftest_bounded_wait(int64_t timeout_ns, void* stream);
+
+/* Thread-local message describing the last non-OK status ("" if none). */
+const char* ck_last_error(void);
+
+/* Library version string. */
+const char* ck_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CK_H_ */

@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every symbol include/ck.h declares, and
+rejects invalid arguments on the host before anything reaches the GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ck():
+    from bit_quantized_linear_rotate_b200 import build
+    build.build()
+    from bit_quantized_linear_rotate_b200 import ck as _ck
+    return _ck
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "ck.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ck_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("ck_rotate_quant_rowwise", "ck_linear_w4a4", "ck_gemv_w4a8", "ck_gemv_awq_w4a16",
+                 "ck_gemm_w4a4", "ck_gemm_w4a4_i32", "ck_gemm_w4a8_i32", "ck_last_error"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(ck):
+    for name in declared_symbols():
+        assert hasattr(ck.lib, name), name
+        assert name in ck.SIGNATURES, f"binding lacks {name}"
+
+
+def test_version_and_last_error(ck):
+    assert "sm_100a" in ck.version()
+    assert isinstance(ck.last_error(), str)
+
+
+def test_workspace_bytes(ck):
+    assert ck.linear_w4a4_workspace_bytes(8192, 3840) == 8192 * 1920 + 8192 * 4
+    assert ck.linear_w4a4_workspace_bytes(3, 64) == 256 + 12
+    assert ck.linear_w4a4_workspace_bytes(0, 64) == 0
+
+
+def _rq(ck, **kw):
+    a = dict(x=1 << 20, xt=0, M=4, K=64, ldx=64, G=64, bits=4, q=1 << 21, s=1 << 22)
+    a.update(kw)
+    p = lambda v: ctypes.c_void_p(v) if v is not None else None
+    return ck.lib.ck_rotate_quant_rowwise(p(a["x"]), a["xt"], a["M"], a["K"], a["ldx"], a["G"], a["bits"],
+                                          p(a["q"]), p(a["s"]), None)
+
+
+def test_rotate_quant_validation(ck):
+    assert _rq(ck, bits=3) == ck.CK_ERR_INVALID_ARG
+    assert _rq(ck, G=48) == ck.CK_ERR_UNSUPPORTED
+    assert _rq(ck, G=512, K=512, ldx=512) == ck.CK_ERR_UNSUPPORTED
+    assert _rq(ck, K=96) == ck.CK_ERR_INVALID_ARG            # K % G != 0
+    assert _rq(ck, ldx=32) == ck.CK_ERR_INVALID_ARG          # ldx < K
+    assert _rq(ck, x=None) == ck.CK_ERR_INVALID_ARG
+    assert _rq(ck, x=(1 << 20) + 2) == ck.CK_ERR_INVALID_ARG  # misaligned rows
+    assert _rq(ck, ldx=68) == ck.CK_ERR_INVALID_ARG          # row stride not 16-byte aligned
+    assert _rq(ck, xt=7) == ck.CK_ERR_INVALID_ARG
+    assert _rq(ck, M=-1) == ck.CK_ERR_INVALID_ARG
+    assert _rq(ck, M=0, x=None, q=None, s=None) == ck.CK_OK  # empty input: no-op
+    assert "bits" in ck.last_error() or True
+
+
+def test_gemm_and_linear_validation(ck):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    assert L.ck_gemm_w4a4(P(1 << 20), P(1 << 20), 8, 48, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemm_w4a4(None, P(1 << 20), 8, 64, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_gemm_w4a4(P(1 << 20), P(1 << 20), 0, 64, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_gemm_w4a4(P((1 << 20) + 8), P(1 << 20), 8, 64, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemm_w4a4_i32(P(1 << 20), P(1 << 20), 8, 64, -1, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_gemm_w4a8_i32(P(1 << 20), None, 8, 64, 8, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    # workspace too small / misaligned
+    assert L.ck_linear_w4a4(P(1 << 20), 0, 8, 64, 8, 64, 64, P(1 << 20), P(1 << 20), None, P(1 << 20),
+                            P(1 << 20), 16, None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_linear_w4a4(P(1 << 20), 0, 8, 64, 8, 64, 64, P(1 << 20), P(1 << 20), None, P(1 << 20),
+                            P((1 << 20) + 16), 1 << 20, None) == ck.CK_ERR_INVALID_ARG
+
+
+def test_gemv_validation(ck):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    assert L.ck_gemv_w4a8(P(1 << 20), P(1 << 20), 17, 128, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemv_w4a8(P(1 << 20), P(1 << 20), 4, 96, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemv_w4a8(P(1 << 20), None, 4, 128, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_gemv_awq_w4a16(P(1 << 20), 0, 9, 128, 8, 64, P(1 << 20), P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemv_awq_w4a16(P(1 << 20), 0, 2, 128, 8, 32, P(1 << 20), P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemv_awq_w4a16(P(1 << 20), 0, 2, 192, 8, 128, P(1 << 20), P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_gemv_awq_w4a16(P(1 << 20), 5, 2, 128, 8, 64, P(1 << 20), P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+
+
+def test_selftest_timeout_range_is_validated(ck):
+    assert ck.lib.ck_selftest_bounded_wait(10, None) == ck.CK_ERR_INVALID_ARG
+    assert ck.lib.ck_selftest_bounded_wait(10 ** 10, None) == ck.CK_ERR_INVALID_ARG
+
+
+def test_package_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "bit_quantized_linear_rotate_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f

@@ -1,0 +1,331 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Small shapes span several tiles and ragged tails; the five workload configs run
+at full size, compared on every output the oracle can afford (all outputs for
+the GEMVs and the M=32 linear, sampled rows for M=8192).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from bit_quantized_linear_rotate_b200 import workloads as WL
+from tests.parity import (assert_codes_close, assert_out_close, assert_scales_close, bf16_tensor_bits,
+                          to_np_f64, unpack_codes)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def ck():
+    from bit_quantized_linear_rotate_b200 import ck as _ck
+    return _ck
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors(ck):
+    yield
+    ck.device_error_check()
+
+
+def _rand_x(M, K, seed, dtype=torch.bfloat16, outliers=0):
+    g = torch.Generator().manual_seed(seed)
+    return WL.activations(M, K, outliers, g, dtype)
+
+
+# ------------------------------------------------------------- rotate_quant
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("G", [16, 64, 256])
+def test_rotate_quant_matches_oracle(ck, G, bits, dtype):
+    M, K = 37, 768
+    xf = _rand_x(M, K + 64, seed=G * 10 + bits, dtype=dtype, outliers=6)
+    x = xf.to(DEV)[:, :K]                       # row stride K + 64: non-contiguous rows
+    q, s = ck.rotate_quant_rowwise(x, G, bits)
+    torch.cuda.synchronize()
+    q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf[:, :K]), G, bits)
+    assert_scales_close(s.cpu().numpy(), s_ref)
+    q_gpu = unpack_codes(q) if bits == 4 else q.cpu().numpy()
+    assert_codes_close(q_gpu, q_ref)
+    if bits == 4:
+        # packed bytes are bit-exact wherever the codes agree
+        same = (O.pack_nibbles(q_ref) == q.cpu().numpy())
+        agree = (q_gpu == q_ref).reshape(M, K // 2, 2).all(axis=2)
+        assert np.array_equal(same[agree], np.ones(int(agree.sum()), dtype=bool))
+
+
+@pytest.mark.parametrize("G", [1, 2, 8, 32, 128])
+def test_rotate_quant_other_group_sizes(ck, G):
+    M, K = 19, 1024
+    xf = _rand_x(M, K, seed=G)
+    q, s = ck.rotate_quant_rowwise(xf.to(DEV), G, 8)
+    q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf), G, 8)
+    assert_scales_close(s.cpu().numpy(), s_ref)
+    assert_codes_close(q.cpu().numpy(), q_ref)
+
+
+def test_rotate_quant_special_rows(ck):
+    G, K = 64, 256
+    x = torch.zeros(6, K)
+    x[1, 70] = 3.0                    # one-hot -> +-qmax Walsh row in group 1
+    x[2, 128:192] = -1.5              # constant group -> [-qmax, 0, ...]
+    x[3] = torch.linspace(-4, 4, K)
+    x[5, 255] = 1e-30                 # tiny but nonzero (bf16 keeps it)
+    xb = x.to(torch.bfloat16)
+    for bits in (4, 8):
+        q, s = ck.rotate_quant_rowwise(xb.to(DEV), G, bits)
+        q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xb), G, bits)
+        q_gpu = unpack_codes(q) if bits == 4 else q.cpu().numpy()
+        assert s.cpu()[0].item() == 1.0 and s.cpu()[4].item() == 1.0      # all-zero rows
+        assert np.all(q_gpu[0] == 0) and np.all(q_gpu[4] == 0)
+        np.testing.assert_array_equal(q_gpu[1], q_ref[1])
+        np.testing.assert_array_equal(q_gpu[2], q_ref[2])
+        assert_scales_close(s.cpu().numpy(), s_ref)
+        assert_codes_close(q_gpu, q_ref, max_frac=1.0 / q_ref.size + 1e-12)
+
+
+def test_rotate_quant_batched_and_empty(ck):
+    xf = _rand_x(10, 512, seed=3).reshape(2, 5, 512)
+    q, s = ck.rotate_quant_rowwise(xf.to(DEV), 64, 4)
+    assert q.shape == (2, 5, 256) and s.shape == (2, 5)
+    q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf.reshape(10, 512)), 64, 4)
+    assert_codes_close(unpack_codes(q.reshape(10, 256)), q_ref)
+    assert_scales_close(s.reshape(10).cpu().numpy(), s_ref)
+    empty = torch.empty(0, 512, device=DEV, dtype=torch.bfloat16)
+    q0, s0 = ck.rotate_quant_rowwise(empty, 64, 4)
+    assert q0.shape == (0, 256) and s0.shape == (0,)
+
+
+@pytest.mark.parametrize("M,K", [(3, 16384), (1500, 32768), (2048, 10240)])
+def test_rotate_quant_long_rows(ck, M, K):
+    xf = _rand_x(M, K, seed=K, outliers=K // 100)
+    q, s = ck.rotate_quant_rowwise(xf.to(DEV), 256, 4)
+    rows = np.unique(np.r_[0, 1, M // 2, M - 1])
+    q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf[rows]), 256, 4)
+    assert_scales_close(s.cpu().numpy()[rows], s_ref)
+    assert_codes_close(unpack_codes(q.cpu()[rows]), q_ref)
+
+
+def test_rotate_quant_mlp_down_G16_full(ck):
+    w = WL.LINEAR_MLP_DOWN
+    x = WL.linear_inputs(w)["x"]
+    for bits in (4, 8):
+        q, s = ck.rotate_quant_rowwise(x.to(DEV), w.rq_group, bits)
+        q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(x), w.rq_group, bits)
+        assert_scales_close(s.cpu().numpy(), s_ref)
+        assert_codes_close(unpack_codes(q) if bits == 4 else q.cpu().numpy(), q_ref)
+
+
+# ------------------------------------------------------- integer GEMM (exact)
+
+GEMM_SHAPES = [(128, 128, 256), (300, 384, 520), (1, 32, 8), (257, 4096, 300), (129, 160, 257),
+               (512, 3840, 768)]
+
+
+@pytest.mark.parametrize("M,K,N", GEMM_SHAPES)
+def test_gemm_w4a4_i32_bit_exact(ck, M, K, N):
+    g = torch.Generator().manual_seed(M * 7 + N)
+    qa = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.uint8)
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    acc = ck.gemm_w4a4_i32(qa.to(DEV), wp.to(DEV))
+    ref = O.int_matmul(O.unpack_nibbles(qa.numpy()), O.unpack_nibbles(wp.numpy()))
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("M,K,N", GEMM_SHAPES)
+def test_gemm_w4a8_i32_bit_exact(ck, M, K, N):
+    g = torch.Generator().manual_seed(M * 11 + N)
+    qa = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    acc = ck.gemm_w4a8_i32(qa.to(DEV), wp.to(DEV))
+    ref = O.int_matmul(qa.numpy().astype(np.int64), O.unpack_nibbles(wp.numpy()))
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref)
+
+
+def test_gemm_extreme_operands(ck):
+    M, K, N = 130, 10240, 260
+    qa = torch.full((M, K // 2), 0xFF, dtype=torch.uint8)      # +7 everywhere
+    wp = torch.zeros((N, K // 2), dtype=torch.uint8)            # -8 everywhere
+    acc = ck.gemm_w4a4_i32(qa.to(DEV), wp.to(DEV)).cpu()
+    assert torch.all(acc == -56 * K)
+    q8 = torch.full((M, K), -127, dtype=torch.int8)
+    acc = ck.gemm_w4a8_i32(q8.to(DEV), wp.to(DEV)).cpu()
+    assert torch.all(acc == 1016 * K)
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("M,K,N", [(200, 512, 300), (128, 3840, 256), (33, 96, 40)])
+def test_gemm_w4a4_epilogue_bit_exact(ck, M, K, N, with_bias):
+    g = torch.Generator().manual_seed(M + N + int(with_bias))
+    qa = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.uint8)
+    sa = (torch.rand(M, generator=g) * 0.5 + 0.01)
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N,), 0.005, 0.02, g)
+    bias = WL.uniform((N,), -1, 1, g) if with_bias else None
+    y = ck.gemm_w4a4(qa.to(DEV), sa.to(DEV), wp.to(DEV), sw.to(DEV), None if bias is None else bias.to(DEV))
+    acc = O.int_matmul(O.unpack_nibbles(qa.numpy()), O.unpack_nibbles(wp.numpy()))
+    ref_bits = O.to_bf16_bits(O.epilogue_rowwise(acc, sa.numpy(), to_np_f64(sw),
+                                                 None if bias is None else to_np_f64(bias)))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), ref_bits)
+
+
+# --------------------------------------------------------- W4A4 linear (e2e)
+
+@pytest.mark.parametrize("M,K,N,G,bias,dtype", [
+    (37, 512, 300, 64, True, torch.bfloat16),
+    (129, 768, 260, 256, False, torch.float16),
+    (300, 256, 520, 16, True, torch.bfloat16),
+    (64, 3840, 3840, 64, False, torch.bfloat16),
+])
+def test_linear_w4a4_matches_oracle(ck, M, K, N, G, bias, dtype):
+    d = WL.small_linear_inputs(M, K, N, seed=M + K, n_outlier_cols=K // 100, dtype=dtype, with_bias=bias)
+    b = d.get("bias")
+    y = ck.linear_w4a4(d["x"].to(DEV), d["w_packed"].to(DEV), d["w_scale"].to(DEV), G,
+                       bias=None if b is None else b.to(DEV))
+    r = O.linear_w4a4(to_np_f64(d["x"]), d["w_packed"].numpy(), to_np_f64(d["w_scale"]), G,
+                      bias=None if b is None else to_np_f64(b))
+    assert_out_close(to_np_f64(y), O.bf16_bits_to_f64(r["y_bits"]))
+
+
+def _linear_full_config(ck, w, sample_rows):
+    d = WL.linear_inputs(w)
+    x, wp, sw = d["x"].to(DEV), d["w_packed"].to(DEV), d["w_scale"].to(DEV)
+    ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=DEV, dtype=torch.uint8)
+    y = ck.linear_w4a4(x, wp, sw, w.G, workspace=ws)
+    torch.cuda.synchronize()
+    rows = np.asarray(sample_rows)
+    r = O.linear_w4a4(to_np_f64(d["x"][rows]), d["w_packed"].numpy(), to_np_f64(d["w_scale"]), w.G)
+    # the quantized activations the GEMM consumed (workspace: packed codes, then scales)
+    nq = w.M * (w.K // 2)
+    qa = ws[:nq].view(w.M, w.K // 2).cpu()[rows]
+    off = (nq + 255) // 256 * 256
+    sa = ws[off:off + 4 * w.M].view(torch.float32).cpu().numpy()[rows]
+    assert_codes_close(unpack_codes(qa), r["q"])
+    assert_scales_close(sa, r["s"])
+    rel = assert_out_close(to_np_f64(y.cpu()[rows]), O.bf16_bits_to_f64(r["y_bits"]))
+    # with identical quantized inputs the GEMM + epilogue is bit-exact
+    acc = O.int_matmul(unpack_codes(qa), O.unpack_nibbles(d["w_packed"].numpy()))
+    exact = O.to_bf16_bits(O.epilogue_rowwise(acc, sa, to_np_f64(d["w_scale"])))
+    np.testing.assert_array_equal(bf16_tensor_bits(y.cpu()[rows]), exact)
+    return rel
+
+
+def test_linear_config_M32_full(ck):
+    _linear_full_config(ck, WL.LINEAR_M32, np.arange(32))
+
+
+def test_linear_config_M8192_sampled(ck):
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.r_[0, 1, 127, 128, 4095, 8190, 8191, rng.integers(0, 8192, 25)])
+    _linear_full_config(ck, WL.LINEAR_M8192, rows)
+
+
+def test_linear_config_mlp_down_sampled(ck):
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.r_[0, 255, 8191, rng.integers(0, 8192, 13)])
+    _linear_full_config(ck, WL.LINEAR_MLP_DOWN, rows)
+
+
+# -------------------------------------------------------------------- GEMVs
+
+def _w4a8_inputs_quantized(w, M):
+    d = WL.gemv_w4a8_inputs(w, M)
+    q, s = O.rotate_quant_rowwise(to_np_f64(d["x"]), 1, 8)     # rowwise int8, no rotation
+    return d, torch.from_numpy(q.astype(np.int8)), torch.from_numpy(s)
+
+
+@pytest.mark.parametrize("M", WL.GEMV_W4A8.Ms)
+def test_gemv_w4a8_config_bit_exact(ck, M):
+    w = WL.GEMV_W4A8
+    d, xq, xs = _w4a8_inputs_quantized(w, M)
+    y = ck.gemv_w4a8(xq.to(DEV), xs.to(DEV), d["w_packed"].to(DEV), d["w_scale"].to(DEV))
+    r = O.gemv_w4a8(xq.numpy(), xs.numpy(), d["w_packed"].numpy(), to_np_f64(d["w_scale"]))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
+
+
+@pytest.mark.parametrize("M,K,N,bias", [(3, 256, 100, True), (9, 512, 37, False), (16, 1280, 48, True),
+                                        (1, 128, 16, False)])
+def test_gemv_w4a8_ragged_bit_exact(ck, M, K, N, bias):
+    g = torch.Generator().manual_seed(M * N)
+    xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    xs = torch.rand(M, generator=g) * 0.1 + 0.001
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N,), 0.005, 0.02, g)
+    b = WL.uniform((N,), -1, 1, g) if bias else None
+    y = ck.gemv_w4a8(xq.to(DEV), xs.to(DEV), wp.to(DEV), sw.to(DEV), None if b is None else b.to(DEV))
+    r = O.gemv_w4a8(xq.numpy(), xs.numpy(), wp.numpy(), to_np_f64(sw), None if b is None else to_np_f64(b))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
+
+
+def test_gemv_w4a8_agrees_with_large_m_gemm(ck):
+    # the decode GEMV and the tensor-core GEMM share codec and epilogue: same int32 results
+    g = torch.Generator().manual_seed(5)
+    M, K, N = 16, 4096, 512
+    xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    ones = torch.ones(M)
+    sw = torch.ones(N, dtype=torch.bfloat16)
+    acc = ck.gemm_w4a8_i32(xq.to(DEV), wp.to(DEV)).cpu()
+    y = ck.gemv_w4a8(xq.to(DEV), ones.to(DEV), wp.to(DEV), sw.to(DEV)).cpu()
+    assert torch.equal(acc.float().to(torch.bfloat16), y)
+
+
+@pytest.mark.parametrize("M", WL.GEMV_AWQ.Ms)
+def test_gemv_awq_config(ck, M):
+    w = WL.GEMV_AWQ
+    d = WL.gemv_awq_inputs(w, M)
+    y = ck.gemv_awq_w4a16(d["x"].to(DEV), d["qweight"].to(DEV), d["wscales"].to(DEV), d["wzeros"].to(DEV),
+                          group_size=w.G)
+    r = O.gemv_awq_w4a16(to_np_f64(d["x"]), d["qweight"].numpy(), to_np_f64(d["wscales"]),
+                         to_np_f64(d["wzeros"]), w.G)
+    assert_out_close(to_np_f64(y), r["y_f64"])
+
+
+@pytest.mark.parametrize("M,K,N,G,dtype,bias", [
+    (1, 128, 40, 64, torch.bfloat16, True),
+    (5, 1024, 70, 128, torch.float16, False),
+    (8, 768, 33, 256, torch.bfloat16, True),
+    (2, 3072, 96, 64, torch.float16, True),
+])
+def test_gemv_awq_variants(ck, M, K, N, G, dtype, bias):
+    g = torch.Generator().manual_seed(K + N)
+    x = WL.activations(M, K, 0, g, dtype)
+    qw = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    ws = WL.uniform((K // G, N), 0.001, 0.01, g, dtype)
+    wz = (torch.randn((K // G, N), generator=g) * 0.01).to(dtype)
+    b = WL.uniform((N,), -1, 1, g, dtype) if bias else None
+    y = ck.gemv_awq_w4a16(x.to(DEV), qw.to(DEV), ws.to(DEV), wz.to(DEV), None if b is None else b.to(DEV),
+                          group_size=G)
+    r = O.gemv_awq_w4a16(to_np_f64(x), qw.numpy(), to_np_f64(ws), to_np_f64(wz), G,
+                         None if b is None else to_np_f64(b))
+    assert_out_close(to_np_f64(y), r["y_f64"])
+
+
+# ------------------------------------------------------------- error paths
+
+def test_bounded_wait_reports_timeout_and_context_survives(ck):
+    ck.selftest_bounded_wait(2_000_000)          # 2 ms: nothing ever arrives
+    with pytest.raises(ck.CKError) as e:
+        ck.device_error_check()
+    assert e.value.status == ck.CK_ERR_TIMEOUT
+    ck.device_error_check()                       # cleared
+    x = _rand_x(4, 256, seed=1).to(DEV)
+    q, s = ck.rotate_quant_rowwise(x, 64, 8)      # the context still works
+    torch.cuda.synchronize()
+    assert torch.all(s > 0)
+
+
+def test_invalid_arguments_raise(ck):
+    x = torch.zeros(4, 96, device=DEV, dtype=torch.bfloat16)
+    with pytest.raises(ck.CKError) as e:
+        ck.rotate_quant_rowwise(x, 64, 4)
+    assert e.value.status == ck.CK_ERR_INVALID_ARG
+    with pytest.raises(ck.CKError) as e:
+        ck.gemv_w4a8(torch.zeros(17, 128, device=DEV, dtype=torch.int8), torch.ones(17, device=DEV),
+                     torch.zeros(8, 64, device=DEV, dtype=torch.uint8), torch.ones(8, device=DEV, dtype=torch.bfloat16))
+    assert e.value.status == ck.CK_ERR_UNSUPPORTED
