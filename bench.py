@@ -195,6 +195,7 @@ def cpu_baseline(w, rows: int):
 # ------------------------------------------------------------------ GPU legs
 
 def time_linear(ck, w, steps: int, warmup: int, world: int, dev):
+    """The linear step as its two C-ABI calls (what ck_linear_w4a4 runs), timed per kernel."""
     d = WL.linear_inputs(w)
     per_copy = d["x"].numel() * 2 + d["w_packed"].numel() + w.M * w.N * 2
     R = max(2, -(-2 * L2_BYTES // per_copy))
@@ -202,21 +203,18 @@ def time_linear(ck, w, steps: int, warmup: int, world: int, dev):
     wps = [d["w_packed"].to(dev) for _ in range(R)]
     sw = d["w_scale"].to(dev)
     ys = [torch.empty(w.M, w.N, device=dev, dtype=torch.bfloat16) for _ in range(R)]
-    nq = w.M * (w.K // 2)
-    ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
-    qa = ws[:nq].view(w.M, w.K // 2)
-    off = (nq + 255) // 256 * 256
-    sa = ws[off:off + 4 * w.M].view(torch.float32)
+    qa = torch.empty(w.M, w.K, device=dev, dtype=torch.int8)
+    sa = torch.empty(w.M, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream()
 
     def step(i, ev=None):
         c = i % R
         if ev is not None:
             ev[0].record(stream)
-        ck.rotate_quant_rowwise(xs[c], w.G, 4, q_out=qa, scale_out=sa)
+        ck.rotate_quant_rowwise_i8(xs[c], w.G, 4, q_out=qa, scale_out=sa)
         if ev is not None:
             ev[1].record(stream)
-        ck.gemm_w4a4(qa, sa, wps[c], sw, out=ys[c])
+        ck.gemm_w4a8(qa, sa, wps[c], sw, out=ys[c])
         if ev is not None:
             ev[2].record(stream)
 
@@ -238,8 +236,19 @@ def time_linear(ck, w, steps: int, warmup: int, world: int, dev):
     total_ms = start.elapsed_time(stop)
     k1 = [e[0].elapsed_time(e[1]) for e in evs]
     k2 = [e[1].elapsed_time(e[2]) for e in evs]
+
+    # the same GEMM with pre-decoded int8 weights (ck_unpack_int4 once, then ck_gemm_s8), and
+    # with packed int4 activations (ck_gemm_w4a4): same outputs, different operand paths
+    w8s = [ck.unpack_int4(wp) for wp in wps]
+    qp, _ = ck.rotate_quant_rowwise(xs[0], w.G, 4)
+    variants = {
+        "gemm_s8_predecoded_us": 1e3 * time_rotating(lambda c: ck.gemm_s8(qa, sa, w8s[c], sw, out=ys[c]), R, 20, 3),
+        "gemm_w4a4_packed_a_us": 1e3 * time_rotating(lambda c: ck.gemm_w4a4(qp, sa, wps[c], sw, out=ys[c]), R, 20, 3),
+        "unpack_int4_us": 1e3 * time_rotating(lambda c: ck.unpack_int4(wps[c], out=w8s[c]), R, 20, 3),
+    }
+    del w8s
     return {"total_ms": total_ms, "k1_ms": statistics.mean(k1), "k2_ms": statistics.mean(k2),
-            "copies": R, "clocks": clk.summary()}
+            "copies": R, "clocks": clk.summary(), "variants": variants}
 
 
 def time_linear_e2e(ck, w, steps: int, warmup: int, dev):
@@ -336,7 +345,7 @@ def run_ours(args, world, rank, local):
     value = ops * world / (ms_step * 1e-3) / 1e12
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
     k2_tops = ops / (t["k2_ms"] * 1e-3) / 1e12
-    k1_bytes = w.M * w.K * 2 + w.M * w.K // 2 + 4 * w.M
+    k1_bytes = w.M * w.K * 2 + w.M * w.K + 4 * w.M       # bf16 in, int8 codes out, scales
     k1_gbs = k1_bytes / (t["k1_ms"] * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world,
@@ -344,7 +353,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
         "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "G": w.G,
-                   "step": "rotate_quant(bits=4) + gemm_w4a4 (bf16 out)",
+                   "step": "ck_rotate_quant_rowwise_i8(bits=4) + ck_gemm_w4a8 (= ck_linear_w4a4)",
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotated over {t['copies']} copies (> 2x L2)"},
         "roofline": {"bound": "tensor", "achieved": round(k2_tops, 1), "peak": round(int8_peak, 1),
@@ -355,7 +364,8 @@ def run_ours(args, world, rank, local):
         "kernels": {"rotate_quant_us": round(t["k1_ms"] * 1e3, 2), "gemm_w4a4_us": round(t["k2_ms"] * 1e3, 2),
                     "rotate_quant_GBps": round(k1_gbs, 1),
                     "rotate_quant_frac_hbm": round(k1_gbs / peaks["hbm_gbs"], 4),
-                    "rotate_quant_traffic": load_traffic("rotate_quant_kernel")},
+                    "rotate_quant_traffic": load_traffic("rotate_quant_kernel"),
+                    **{k: round(v, 2) for k, v in t["variants"].items()}},
         "gpu_launches": 2 * args.steps,
         "clocks": t["clocks"],
     }

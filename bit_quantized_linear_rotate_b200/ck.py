@@ -36,7 +36,12 @@ _int = ctypes.c_int
 # name -> argument types (restype is ck_status = int unless listed below)
 SIGNATURES = {
     "ck_rotate_quant_rowwise": [_p, _int, _i64, _i64, _i64, _int, _int, _p, _p, _p],
+    "ck_rotate_quant_rowwise_i8": [_p, _int, _i64, _i64, _i64, _int, _int, _p, _p, _p],
     "ck_gemm_w4a4": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+    "ck_gemm_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+    "ck_unpack_int4": [_p, _i64, _i64, _p, _p],
+    "ck_gemm_s8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+    "ck_gemm_s8_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
     "ck_linear_w4a4_workspace_bytes": [_i64, _i64],
     "ck_linear_w4a4": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
     "ck_gemv_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
@@ -127,6 +132,65 @@ def rotate_quant_rowwise(x, group_size: int, bits: int, q_out=None, scale_out=No
                                        _ptr(q_out), _ptr(scale_out), _stream(stream)),
            "ck_rotate_quant_rowwise")
     return q_out, scale_out
+
+
+def rotate_quant_rowwise_i8(x, group_size: int, bits: int, q_out=None, scale_out=None, stream=None):
+    """Returns (q, scale) with the codes stored one per byte: q (..., K) int8 for bits 4 or 8."""
+    _cuda(x)
+    M, K, ldx, x2 = _rows(x)
+    lead = tuple(x.shape[:-1])
+    if q_out is None:
+        q_out = torch.empty(lead + (K,), device=x.device, dtype=torch.int8)
+    if scale_out is None:
+        scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
+    _cuda(q_out, scale_out)
+    _check(lib.ck_rotate_quant_rowwise_i8(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
+                                          _ptr(q_out), _ptr(scale_out), _stream(stream)),
+           "ck_rotate_quant_rowwise_i8")
+    return q_out, scale_out
+
+
+def unpack_int4(packed, out=None, stream=None):
+    """(R, C/2) packed int4 -> (R, C) int8 with value u - 8."""
+    _cuda(packed)
+    R, Ch = packed.shape
+    if out is None:
+        out = torch.empty((R, 2 * Ch), device=packed.device, dtype=torch.int8)
+    _check(lib.ck_unpack_int4(_ptr(packed), R, 2 * Ch, _ptr(out), _stream(stream)), "ck_unpack_int4")
+    return out
+
+
+def gemm_w4a8(qa, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):
+    """int8 activation codes (M, K) x packed int4 weights (N, K/2) -> bf16 (M, N)."""
+    _cuda(qa, a_scale, w_packed, w_scale, bias)
+    M, K = qa.shape
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=qa.device, dtype=torch.bfloat16)
+    _check(lib.ck_gemm_w4a8(_ptr(qa), _ptr(a_scale), M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias),
+                            _ptr(out), _stream(stream)), "ck_gemm_w4a8")
+    return out
+
+
+def gemm_s8(qa, a_scale, w8, w_scale, bias=None, out=None, stream=None):
+    _cuda(qa, a_scale, w8, w_scale, bias)
+    M, K = qa.shape
+    N = w8.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=qa.device, dtype=torch.bfloat16)
+    _check(lib.ck_gemm_s8(_ptr(qa), _ptr(a_scale), M, K, N, _ptr(w8), _ptr(w_scale), _ptr(bias), _ptr(out),
+                          _stream(stream)), "ck_gemm_s8")
+    return out
+
+
+def gemm_s8_i32(qa, w8, out=None, stream=None):
+    _cuda(qa, w8)
+    M, K = qa.shape
+    N = w8.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=qa.device, dtype=torch.int32)
+    _check(lib.ck_gemm_s8_i32(_ptr(qa), _ptr(w8), M, K, N, _ptr(out), _stream(stream)), "ck_gemm_s8_i32")
+    return out
 
 
 def gemm_w4a4(qa_packed, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):

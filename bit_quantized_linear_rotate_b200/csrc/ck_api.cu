@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -100,40 +101,31 @@ ck_status ensure_smem_attr(KernelT kernel, size_t bytes) {
   return CK_OK;
 }
 
-template <int VPT, int BITS, typename T>
+template <int QBITS, int STORE, typename T>
 void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s, int nt,
                cudaStream_t st) {
   const float rnorm = (float)(1.0 / std::sqrt((double)G));
-  ck::rq::rotate_quant_kernel<VPT, BITS, T><<<(unsigned)M, nt, 0, st>>>(
+  ck::rq::rotate_quant_kernel<QBITS, STORE, T><<<(unsigned)M, nt, 0, st>>>(
       reinterpret_cast<const T*>(x), K, ldx, G, rnorm, reinterpret_cast<uint8_t*>(q), s);
 }
 
-template <int BITS, typename T>
-void launch_rq_vpt(int vpt, const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s,
-                   int nt, cudaStream_t st) {
-  switch (vpt) {
-    case 1: launch_rq<1, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
-    case 2: launch_rq<2, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
-    case 4: launch_rq<4, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
-    default: launch_rq<8, BITS, T>(x, M, K, ldx, G, q, s, nt, st); break;
-  }
-}
-
+// store: ck::rq::STORE_PACKED4 (bits must be 4) or ck::rq::STORE_INT8 (codes as int8 bytes).
 ck_status rotate_quant_impl(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int G,
-                            int bits, void* q, float* s, cudaStream_t st) {
-  const int64_t nvec = K / 8;
-  const int target = M >= 1024 ? 128 : 1024;
-  int vpt = 1;
-  while (vpt < 8 && (nvec + vpt - 1) / vpt > target) vpt *= 2;
-  int64_t nt = ((nvec + vpt - 1) / vpt + 31) / 32 * 32;
-  if (nt > ck::rq::max_threads(vpt))
-    return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K=%lld too large (max 32768)", (long long)K);
+                            int bits, int store, void* q, float* s, cudaStream_t st) {
+  using namespace ck::rq;
+  const int64_t nt = ((K + EPT - 1) / EPT + 31) / 32 * 32;
+  if (nt > 1024) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K=%lld too large (max 32768)", (long long)K);
+  const int k = (int)K, n = (int)nt;
   if (xt == CK_BF16) {
-    if (bits == 4) launch_rq_vpt<4, __nv_bfloat16>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
-    else launch_rq_vpt<8, __nv_bfloat16>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
+    using T = __nv_bfloat16;
+    if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, k, ldx, G, q, s, n, st);
+    else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
+    else launch_rq<8, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
   } else {
-    if (bits == 4) launch_rq_vpt<4, __half>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
-    else launch_rq_vpt<8, __half>(vpt, x, M, (int)K, ldx, G, q, s, (int)nt, st);
+    using T = __half;
+    if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, k, ldx, G, q, s, n, st);
+    else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
+    else launch_rq<8, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
   }
   return launch_status("rotate_quant");
 }
@@ -148,21 +140,23 @@ ck_status check_gemm_shape(const char* who, int64_t M, int64_t K, int64_t N) {
   return CK_OK;
 }
 
-template <bool A_PACKED, int EPI>
-ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const uint8_t* w,
+template <int A_MODE, int B_MODE, int EPI>
+ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const void* w,
                     const float* a_scale, const uint16_t* w_scale, const uint16_t* bias, void* out,
                     cudaStream_t st) {
   using namespace ck::gemm;
+  using C = Cfg<A_MODE, B_MODE>;
   CUtensorMap ta, tb;
   ck_status r;
-  if (A_PACKED) r = make_tmap(&ta, qa, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, PKB, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (C::AP) r = make_tmap(&ta, qa, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, PKB, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
   else r = make_tmap(&ta, qa, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (r != CK_OK) return r;
-  r = make_tmap(&tb, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, PKB, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (C::BP) r = make_tmap(&tb, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, PKB, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else r = make_tmap(&tb, w, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (r != CK_OK) return r;
-  auto kern = gemm_w4_kernel<A_PACKED, EPI>;
+  auto kern = gemm_w4_kernel<A_MODE, B_MODE, EPI>;
   struct Tag {};
-  if ((r = ensure_smem_attr<Tag>(kern, kSmemBytes)) != CK_OK) return r;
+  if ((r = ensure_smem_attr<Tag>(kern, C::SMEM)) != CK_OK) return r;
   Params p;
   p.M = (int)M; p.N = (int)N; p.K = (int)K;
   p.a_scale = a_scale;
@@ -172,9 +166,11 @@ ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const uint8
   const size_t esz = EPI == EPI_I32 ? 4 : 2;
   p.out_vec_ok = aligned(out, 16) && ((N * (int64_t)esz) % 16 == 0);
   dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-  kern<<<grid, kThreads, kSmemBytes, st>>>(ta, tb, p);
+  kern<<<grid, kThreads, C::SMEM, st>>>(ta, tb, p);
   return launch_status("gemm_w4");
 }
+
+size_t linear_q_bytes(int64_t M, int64_t K) { return ((size_t)M * (size_t)K + 255) / 256 * 256; }
 
 }  // namespace
 
@@ -201,7 +197,76 @@ ck_status ck_rotate_quant_rowwise(const void* x, ck_dtype xt, int64_t M, int64_t
   if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant: x rows must be 16-byte aligned");
   if (!aligned(q_out, 16) || !aligned(scale_out, 4)) return fail(CK_ERR_INVALID_ARG, "rotate_quant: misaligned output");
   if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: M too large");
-  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, q_out, scale_out, S(stream));
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits,
+                           bits == 4 ? ck::rq::STORE_PACKED4 : ck::rq::STORE_INT8, q_out, scale_out,
+                           S(stream));
+}
+
+ck_status ck_rotate_quant_rowwise_i8(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                     int group_size, int bits, int8_t* q_out, float* scale_out,
+                                     void* stream) {
+  if (M < 0 || K <= 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: need M >= 0 and K > 0");
+  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: unknown dtype");
+  if (bits != 4 && bits != 8) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: bits must be 4 or 8");
+  if (!is_pow2(group_size) || group_size > 256)
+    return fail(CK_ERR_UNSUPPORTED, "rotate_quant_i8: group_size=%d must be a power of two <= 256", group_size);
+  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: K %% group_size != 0");
+  if (K % 8 != 0) return fail(CK_ERR_UNSUPPORTED, "rotate_quant_i8: K must be a multiple of 8");
+  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: ldx < K");
+  if (M == 0) return ok();
+  if (x == nullptr || q_out == nullptr || scale_out == nullptr)
+    return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: null pointer");
+  if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: x rows must be 16-byte aligned");
+  if (!aligned(q_out, 16) || !aligned(scale_out, 4)) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: misaligned output");
+  if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "rotate_quant_i8: M too large");
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, ck::rq::STORE_INT8, q_out, scale_out, S(stream));
+}
+
+ck_status ck_unpack_int4(const uint8_t* packed, int64_t R, int64_t C, int8_t* out, void* stream) {
+  if (R <= 0 || C <= 0) return fail(CK_ERR_INVALID_ARG, "unpack_int4: R, C must be > 0");
+  if (!packed || !out) return fail(CK_ERR_INVALID_ARG, "unpack_int4: null pointer");
+  const int64_t nbytes = R * (C / 2);
+  if (C % 2 != 0 || nbytes % 16 != 0) return fail(CK_ERR_UNSUPPORTED, "unpack_int4: R*C/2 must be a multiple of 16");
+  if (!aligned(packed, 16) || !aligned(out, 16)) return fail(CK_ERR_INVALID_ARG, "unpack_int4: pointers must be 16-byte aligned");
+  const int64_t n16 = nbytes / 16;
+  const unsigned grid = (unsigned)std::min<int64_t>((n16 + 255) / 256, 148 * 16);
+  ck::gemm::unpack_int4_kernel<<<grid, 256, 0, S(stream)>>>(reinterpret_cast<const uint4*>(packed),
+                                                            reinterpret_cast<uint4*>(out), n16);
+  return launch_status("unpack_int4");
+}
+
+ck_status ck_gemm_s8(const int8_t* qa, const float* a_scale, int64_t M, int64_t K, int64_t N,
+                     const int8_t* w, const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                     void* stream) {
+  ck_status r = check_gemm_shape("gemm_s8", M, K, N);
+  if (r != CK_OK) return r;
+  if (!qa || !a_scale || !w || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemm_s8: null pointer");
+  if (!aligned(qa, 16) || !aligned(w, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_s8: operands must be 16-byte aligned");
+  if (!aligned(a_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "gemm_s8: misaligned scale, bias or output");
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_BF16>(qa, M, K, N, w, a_scale, w_scale, bias, y, S(stream));
+}
+
+ck_status ck_gemm_w4a8(const int8_t* qa, const float* a_scale, int64_t M, int64_t K, int64_t N,
+                       const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
+                       uint16_t* y, void* stream) {
+  ck_status r = check_gemm_shape("gemm_w4a8", M, K, N);
+  if (r != CK_OK) return r;
+  if (!qa || !a_scale || !w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8: null pointer");
+  if (!aligned(qa, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a8: operands must be 16-byte aligned");
+  if (!aligned(a_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "gemm_w4a8: misaligned scale, bias or output");
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4, ck::gemm::EPI_BF16>(qa, M, K, N, w_packed, a_scale, w_scale, bias, y, S(stream));
+}
+
+ck_status ck_gemm_s8_i32(const int8_t* qa, const int8_t* w, int64_t M, int64_t K, int64_t N, int32_t* acc,
+                         void* stream) {
+  ck_status r = check_gemm_shape("gemm_s8_i32", M, K, N);
+  if (r != CK_OK) return r;
+  if (!qa || !w || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_s8_i32: null pointer");
+  if (!aligned(qa, 16) || !aligned(w, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_s8_i32: operands must be 16-byte aligned");
+  if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_s8_i32: misaligned output");
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_I32>(qa, M, K, N, w, nullptr, nullptr, nullptr, acc, S(stream));
 }
 
 ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M, int64_t K,
@@ -213,13 +278,12 @@ ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M
   if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4: operands must be 16-byte aligned");
   if (!aligned(a_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "gemm_w4a4: misaligned scale, bias or output");
-  return gemm_impl<true, ck::gemm::EPI_BF16>(qa_packed, M, K, N, w_packed, a_scale, w_scale, bias, y, S(stream));
+  return gemm_impl<ck::gemm::OP_PACKED4, ck::gemm::OP_PACKED4, ck::gemm::EPI_BF16>(qa_packed, M, K, N, w_packed, a_scale, w_scale, bias, y, S(stream));
 }
 
 size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K) {
   if (M <= 0 || K <= 0) return 0;
-  const size_t qa = ((size_t)M * (size_t)(K / 2) + 255) / 256 * 256;
-  return qa + (size_t)M * sizeof(float);
+  return linear_q_bytes(M, K) + (size_t)M * sizeof(float);
 }
 
 ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
@@ -235,11 +299,12 @@ ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64
   if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "linear_w4a4: weights must be 16-byte aligned");
   if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "linear_w4a4: misaligned scale, bias or output");
-  uint8_t* qa = reinterpret_cast<uint8_t*>(workspace);
-  float* sa = reinterpret_cast<float*>(qa + ((size_t)M * (size_t)(K / 2) + 255) / 256 * 256);
-  r = ck_rotate_quant_rowwise(x, xt, M, K, ldx, group_size, 4, qa, sa, stream);
+  // int4 codes (|q| <= 7) stored one per byte: the GEMM reads them with TMA, no activation unpack
+  int8_t* qa = reinterpret_cast<int8_t*>(workspace);
+  float* sa = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + linear_q_bytes(M, K));
+  r = ck_rotate_quant_rowwise_i8(x, xt, M, K, ldx, group_size, 4, qa, sa, stream);
   if (r != CK_OK) return r;
-  return gemm_impl<true, ck::gemm::EPI_BF16>(qa, M, K, N, w_packed, sa, w_scale, bias, y, S(stream));
+  return ck_gemm_w4a8(qa, sa, M, K, N, w_packed, w_scale, bias, y, stream);
 }
 
 ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, int64_t M, int64_t K,
@@ -249,7 +314,7 @@ ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, in
   if (!qa_packed || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4_i32: null pointer");
   if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4_i32: operands must be 16-byte aligned");
   if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4_i32: misaligned output");
-  return gemm_impl<true, ck::gemm::EPI_I32>(qa_packed, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
+  return gemm_impl<ck::gemm::OP_PACKED4, ck::gemm::OP_PACKED4, ck::gemm::EPI_I32>(qa_packed, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
 }
 
 ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M, int64_t K, int64_t N,
@@ -259,7 +324,7 @@ ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M,
   if (!qa || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8_i32: null pointer");
   if (!aligned(qa, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a8_i32: operands must be 16-byte aligned");
   if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8_i32: misaligned output");
-  return gemm_impl<false, ck::gemm::EPI_I32>(qa, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4, ck::gemm::EPI_I32>(qa, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
 }
 
 ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,

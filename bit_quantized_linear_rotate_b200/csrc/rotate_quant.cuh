@@ -2,19 +2,21 @@
 //
 // Follows "quantize_and_rotate_rowwise" (comfy-kitchen PR #155 "[Feat][Ascend]
 // Add fused RotateQuant backend", "What this PR does": group rotation, rowwise
-// dynamic quantization, positive scale, zero-row handling) with the
-// warp-shuffle Hadamard transform named in comfy-kitchen PR #182
-// ("Description": the CUDA INT8 rowwise ConvRot quantizer of #176).
+// dynamic quantization, positive scale, zero-row handling) with a register /
+// warp-shuffle Hadamard transform as in the CUDA INT8 rowwise ConvRot quantizer
+// named by comfy-kitchen PR #182 ("Description").
 //
-// One CTA per row. Thread t owns 8-element vectors v = i * blockDim + t
-// (i < VPT) loaded with 128-bit loads, so a warp covers 256 consecutive
-// columns per iteration and every Hadamard group (G <= 256 columns = G/8
-// vectors) sits in G/8 consecutive lanes. The transform runs in fp32:
-// three butterfly stages inside the thread, log2(G/8) stages across lanes
-// with __shfl_xor_sync, then the 1/sqrt(G) normalisation (exact for G = 16,
-// 64, 256). The rotated row never leaves registers: amax is reduced across the
-// CTA, then each thread quantizes and stores its own values (4 bytes of packed
-// int4 or 8 bytes of int8 per vector, coalesced across the warp).
+// One CTA per row; thread t owns the 32 contiguous columns [32t, 32t + 32)
+// (four 128-bit loads). The transform runs in fp32: log2(min(G, 32)) butterfly
+// stages inside the thread, then log2(G / 32) stages across lanes
+// (__shfl_xor_sync, one shuffle and one FMA per element and stage), then the
+// 1/sqrt(G) normalisation (a power of two for G = 16, 64, 256). The rotated row
+// never leaves registers: amax is reduced across the CTA, then every thread
+// quantizes its 32 values and writes 16 bytes (packed int4) or 32 bytes (int8).
+//
+// Quantization multiplies by the reciprocal of the scale; when the product lies
+// within 1e-4 of a rounding boundary it is recomputed with the correctly
+// rounded quotient y / s, so ties are decided as by division.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,11 +27,15 @@
 namespace ck {
 namespace rq {
 
+constexpr int EPT = 32;   // columns per thread
+
+enum Store { STORE_PACKED4 = 0, STORE_INT8 = 1 };
+
 template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&f)[8]);
+__device__ __forceinline__ void load8(const T* p, float* f);
 
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&f)[8]) {
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
   const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(p));
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -40,7 +46,7 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
 }
 
 template <>
-__device__ __forceinline__ void load8<__half>(const __half* p, float (&f)[8]) {
+__device__ __forceinline__ void load8<__half>(const __half* p, float* f) {
   const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(p));
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -51,14 +57,14 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float (&f)[8]) {
   }
 }
 
-// y[e] for e in 0..7 -> Sylvester butterflies on element-index bits 0..2 (only
-// the bits below G). Index bit b set => new = x(bit clear) - x(bit set).
-__device__ __forceinline__ void fht_in_thread(float (&v)[8], int G) {
+// Sylvester butterflies on element-index bits below min(G, 32): for index bit h,
+// (a, b) -> (a + b, a - b) where a has the bit clear.
+__device__ __forceinline__ void fht_in_thread(float (&v)[EPT], int G) {
 #pragma unroll
-  for (int h = 1; h < 8; h <<= 1) {
+  for (int h = 1; h < EPT; h <<= 1) {
     if (h < G) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < EPT; ++e) {
         if ((e & h) == 0) {
           const float a = v[e], b = v[e + h];
           v[e] = a + b;
@@ -69,61 +75,57 @@ __device__ __forceinline__ void fht_in_thread(float (&v)[8], int G) {
   }
 }
 
-// Stages on element-index bits 3.. (lane bits 0..): partner lane = lane ^ j.
-__device__ __forceinline__ void fht_across_lanes(float (&v)[8], int G, int lane) {
-  for (int j = 1; 8 * j < G; j <<= 1) {
-    const bool upper = (lane & j) != 0;
+// Index bits 5.. live in lane bits 0..: new = partner + v (bit clear) or partner - v (bit set).
+__device__ __forceinline__ void fht_across_lanes(float (&v)[EPT], int G, int lane) {
+  for (int j = 1; EPT * j < G; j <<= 1) {
+    const float sgn = (lane & j) ? -1.0f : 1.0f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < EPT; ++e) {
       const float other = __shfl_xor_sync(0xffffffffu, v[e], j);
-      v[e] = upper ? (other - v[e]) : (v[e] + other);
+      v[e] = fmaf(sgn, v[e], other);
     }
   }
 }
 
-// Threads per CTA allowed for VPT vectors per thread (keeps VPT = 8 in registers).
-__host__ __device__ constexpr int max_threads(int vpt) { return vpt >= 8 ? 512 : 1024; }
+__device__ __forceinline__ int quant1(float y, float r, float s, float qmax) {
+  float t = __fmul_rn(y, r);
+  const float f = t - truncf(t);
+  if (fabsf(fabsf(f) - 0.5f) < 1e-4f) t = __fdiv_rn(y, s);
+  return (int)fminf(fmaxf(rintf(t), -qmax), qmax);
+}
 
-template <int VPT, int BITS, typename T>
-__global__ void __launch_bounds__(max_threads(VPT)) rotate_quant_kernel(const T* __restrict__ x, int K,
-                                                            int64_t ldx, int G, float rnorm,
-                                                            uint8_t* __restrict__ q,
+template <int QBITS, int STORE, typename T>
+__global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict__ x, int K, int64_t ldx,
+                                                            int G, float rnorm, uint8_t* __restrict__ q,
                                                             float* __restrict__ scale) {
-  constexpr float kQmax = BITS == 4 ? 7.0f : 127.0f;
+  constexpr float kQmax = QBITS == 4 ? 7.0f : 127.0f;
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
-  const int nvec = K >> 3;
+  const int e0 = tid * EPT;
   const T* xr = x + row * ldx;
 
-  float v[VPT][8];
+  float v[EPT];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int vi = i * blockDim.x + tid;
-    if (vi < nvec) {
-      load8<T>(xr + 8 * vi, v[i]);
+  for (int j = 0; j < EPT / 8; ++j) {
+    if (e0 + 8 * j < K) {
+      load8<T>(xr + e0 + 8 * j, v + 8 * j);
     } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[i][e] = 0.0f;
+      for (int e = 0; e < 8; ++e) v[8 * j + e] = 0.0f;
     }
   }
 
+  if (G > 1) {
+    fht_in_thread(v, G);
+    fht_across_lanes(v, G, lane);   // every lane runs it; columns past K hold zeros
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) v[e] *= rnorm;
+  }
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    // every lane of the warp runs the shuffles; vectors past the row are zeros
-    if (i * (int)blockDim.x < nvec) {
-      if (G > 1) {
-        fht_in_thread(v[i], G);
-        fht_across_lanes(v[i], G, lane);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[i][e] *= rnorm;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
-    }
-  }
+  for (int e = 0; e < EPT; ++e) amax = fmaxf(amax, fabsf(v[e]));
 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -142,31 +144,43 @@ __global__ void __launch_bounds__(max_threads(VPT)) rotate_quant_kernel(const T*
   const float s = amax > 0.0f ? __fdiv_rn(amax, kQmax) : 1.0f;
   const float r = __frcp_rn(s);
   if (tid == 0) scale[row] = s;
+  if (e0 >= K) return;
 
+  if (STORE == STORE_PACKED4) {
+    // 32 codes -> 16 bytes, u = q + 8, low nibble = even column
+    uint32_t w[4];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int vi = i * blockDim.x + tid;
-    if (vi < nvec) {
-      int qi[8];
+    for (int j = 0; j < 4; ++j) {
+      uint32_t acc = 0;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float t = rintf(__fmul_rn(v[i][e], r));
-        qi[e] = (int)fminf(fmaxf(t, -kQmax), kQmax);
-      }
-      if (BITS == 4) {
-        uint32_t packed = 0;
+      for (int e = 0; e < 8; ++e) acc |= (uint32_t)(quant1(v[8 * j + e], r, s, kQmax) + 8) << (4 * e);
+      w[j] = acc;
+    }
+    uint8_t* qr = q + row * (int64_t)(K >> 1) + (e0 >> 1);
+    if ((K & 31) == 0) {          // rows of K/2 bytes are 16-byte aligned
+      *reinterpret_cast<uint4*>(qr) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) packed |= (uint32_t)(qi[e] + 8) << (4 * e);
-        reinterpret_cast<uint32_t*>(q + row * (int64_t)(K >> 1))[vi] = packed;
-      } else {
-        uint32_t lo = 0, hi = 0;
+      for (int j = 0; j < 4; ++j)
+        if (e0 + 8 * j < K) reinterpret_cast<uint32_t*>(qr)[j] = w[j];
+    }
+  } else {
+    uint32_t w[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          lo |= (uint32_t)(qi[e] & 0xFF) << (8 * e);
-          hi |= (uint32_t)(qi[e + 4] & 0xFF) << (8 * e);
-        }
-        reinterpret_cast<uint2*>(q + row * (int64_t)K)[vi] = make_uint2(lo, hi);
-      }
+    for (int j = 0; j < 8; ++j) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc |= (uint32_t)(quant1(v[4 * j + e], r, s, kQmax) & 0xFF) << (8 * e);
+      w[j] = acc;
+    }
+    uint8_t* qr = q + row * (int64_t)K + e0;
+    if ((K & 31) == 0) {
+      reinterpret_cast<uint4*>(qr)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(qr)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (e0 + 8 * j < K) reinterpret_cast<uint2*>(qr)[j] = make_uint2(w[2 * j], w[2 * j + 1]);
     }
   }
 }

@@ -69,6 +69,18 @@ ck_status ck_rotate_quant_rowwise(const void* x, ck_dtype xt, int64_t M, int64_t
                                   float* scale_out, void* stream);
 
 /*
+ * Same rotation and quantization as ck_rotate_quant_rowwise, with the codes
+ * stored one per byte: q_out is (M, K) int8 for bits = 4 (|q| <= 7) as well as
+ * bits = 8 (|q| <= 127). This is the activation format the W4A4 linear feeds
+ * its GEMM (comfy-kitchen PR #212 "Related work": PR #201 removes the
+ * activation pack/unpack); the int4 code values are identical to the packed
+ * output's.
+ */
+ck_status ck_rotate_quant_rowwise_i8(const void* x, ck_dtype xt, int64_t M, int64_t K,
+                                     int64_t ldx, int group_size, int bits, int8_t* q_out,
+                                     float* scale_out, void* stream);
+
+/*
  * Integer matmul of packed int4 activations with packed int4 weights, int32
  * accumulation on the tcgen05 tensor cores, and the rowwise-scale epilogue
  * (the "EpiRowwise" of comfy-kitchen PR #182, Description):
@@ -89,13 +101,45 @@ ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M
                        int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
                        const uint16_t* bias, uint16_t* y, void* stream);
 
+/*
+ * Large-M W4A8 GEMM ("asym_w4a8_int8", stable-diffusion.cpp PR #2276,
+ * Summary): int8 activation codes times packed int4 weights, the same main
+ * loop and epilogue as ck_gemm_w4a4 with the activation tile loaded by TMA
+ * instead of decoded. ck_linear_w4a4 runs exactly ck_rotate_quant_rowwise_i8
+ * (bits=4) followed by this call.
+ * qa (M, K) int8 (any codes in [-127, 127]), 16-byte aligned; K % 32 == 0.
+ */
+ck_status ck_gemm_w4a8(const int8_t* qa, const float* a_scale, int64_t M, int64_t K, int64_t N,
+                       const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
+                       uint16_t* y, void* stream);
+
+/*
+ * Unpacks a packed int4 matrix (R, C/2) into int8 (R, C) with value u - 8: the
+ * weight preparation that comfy-kitchen PR #212 ("Summary", "Memory and support
+ * limits") caches across calls, as a standalone pass the caller can run once.
+ * Requires C even, R*C/2 a multiple of 16 and 16-byte aligned pointers.
+ */
+ck_status ck_unpack_int4(const uint8_t* packed, int64_t R, int64_t C, int8_t* out, void* stream);
+
+/*
+ * ck_gemm_w4a4 with both operands already int8 (activation codes from
+ * ck_rotate_quant_rowwise_i8, weights from ck_unpack_int4): the pre-decoded
+ * weight variant, trading twice the weight bytes for no in-kernel decode.
+ * qa (M, K) int8, w (N, K) int8, both 16-byte aligned; K % 32 == 0.
+ */
+ck_status ck_gemm_s8(const int8_t* qa, const float* a_scale, int64_t M, int64_t K, int64_t N,
+                     const int8_t* w, const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                     void* stream);
+
 /* Bytes of device workspace ck_linear_w4a4 needs for M rows of logical width K. */
 size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K);
 
 /*
  * The ConvRot W4A4 linear ("public ConvRot W4A4 Linear dispatcher",
  * comfy-kitchen PR #212; packed formats of stable-diffusion.cpp PR #2276):
- * ck_rotate_quant_rowwise(bits=4) into `workspace`, then ck_gemm_w4a4.
+ * ck_rotate_quant_rowwise_i8(bits=4) into `workspace`, then the GEMM of
+ * ck_gemm_w4a4 reading those int8 codes against the packed int4 weights (same
+ * results as ck_rotate_quant_rowwise + ck_gemm_w4a4).
  * K is the LOGICAL inner dimension (the packed weight has K/2 bytes per row).
  * workspace : device buffer of at least ck_linear_w4a4_workspace_bytes(M, K)
  *             bytes, 256-byte aligned; its contents are scratch.
@@ -146,6 +190,9 @@ ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, in
                            int64_t K, int64_t N, int32_t* acc, void* stream);
 ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M, int64_t K,
                            int64_t N, int32_t* acc, void* stream);
+/* Test hook of ck_gemm_s8: int8 activations and int8 weights -> int32. */
+ck_status ck_gemm_s8_i32(const int8_t* qa, const int8_t* w, int64_t M, int64_t K, int64_t N,
+                         int32_t* acc, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device error word set by a

@@ -27,6 +27,7 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ("ck_rotate_quant_rowwise", "ck_linear_w4a4", "ck_gemv_w4a8", "ck_gemv_awq_w4a16",
+                 "ck_rotate_quant_rowwise_i8", "ck_gemm_w4a8", "ck_unpack_int4", "ck_gemm_s8",
                  "ck_gemm_w4a4", "ck_gemm_w4a4_i32", "ck_gemm_w4a8_i32", "ck_last_error"):
         assert name in syms
 
@@ -43,7 +44,8 @@ def test_version_and_last_error(ck):
 
 
 def test_workspace_bytes(ck):
-    assert ck.linear_w4a4_workspace_bytes(8192, 3840) == 8192 * 1920 + 8192 * 4
+    # int8 activation codes (rounded up to 256 bytes), then float32 scales
+    assert ck.linear_w4a4_workspace_bytes(8192, 3840) == 8192 * 3840 + 8192 * 4
     assert ck.linear_w4a4_workspace_bytes(3, 64) == 256 + 12
     assert ck.linear_w4a4_workspace_bytes(0, 64) == 0
 
@@ -85,6 +87,20 @@ def test_gemm_and_linear_validation(ck):
                             P(1 << 20), 16, None) == ck.CK_ERR_INVALID_ARG
     assert L.ck_linear_w4a4(P(1 << 20), 0, 8, 64, 8, 64, 64, P(1 << 20), P(1 << 20), None, P(1 << 20),
                             P((1 << 20) + 16), 1 << 20, None) == ck.CK_ERR_INVALID_ARG
+
+
+def test_predecoded_path_validation(ck):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    assert L.ck_unpack_int4(P(1 << 20), 3, 6, P(1 << 21), None) == ck.CK_ERR_UNSUPPORTED   # 9 bytes
+    assert L.ck_unpack_int4(P(1 << 20), 4, 7, P(1 << 21), None) == ck.CK_ERR_UNSUPPORTED   # odd C
+    assert L.ck_unpack_int4(None, 4, 8, P(1 << 21), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_unpack_int4(P((1 << 20) + 4), 4, 8, P(1 << 21), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_gemm_s8(P(1 << 20), P(1 << 20), 8, 40, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemm_w4a8(P(1 << 20), None, 8, 64, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_gemm_s8_i32(P(1 << 20), P(1 << 20), 8, 64, 0, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_rotate_quant_rowwise_i8(P(1 << 20), 0, 4, 64, 64, 64, 5, P(1 << 21), P(1 << 22), None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_rotate_quant_rowwise_i8(P(1 << 20), 0, 4, 64, 64, 3, 4, P(1 << 21), P(1 << 22), None) == ck.CK_ERR_UNSUPPORTED
 
 
 def test_gemv_validation(ck):

@@ -121,6 +121,30 @@ def test_rotate_quant_mlp_down_G16_full(ck):
         assert_codes_close(unpack_codes(q) if bits == 4 else q.cpu().numpy(), q_ref)
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("G,K", [(64, 3840), (16, 1000), (256, 512)])
+def test_rotate_quant_i8_codes_equal_packed_codes(ck, G, K, bits):
+    M = 70
+    xf = _rand_x(M, K, seed=K + bits, outliers=3)
+    x = xf.to(DEV)
+    q8, s8 = ck.rotate_quant_rowwise_i8(x, G, bits)
+    q, s = ck.rotate_quant_rowwise(x, G, bits)
+    q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf), G, bits)
+    assert torch.equal(s8, s)
+    q_other = unpack_codes(q) if bits == 4 else q.cpu().numpy()
+    np.testing.assert_array_equal(q8.cpu().numpy(), q_other)
+    assert_codes_close(q8.cpu().numpy(), q_ref)
+    assert_scales_close(s8.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("R,C", [(3840, 3840), (7, 64), (1, 32)])
+def test_unpack_int4_bit_exact(ck, R, C):
+    g = torch.Generator().manual_seed(R + C)
+    wp = torch.randint(0, 256, (R, C // 2), generator=g, dtype=torch.uint8)
+    w8 = ck.unpack_int4(wp.to(DEV))
+    np.testing.assert_array_equal(w8.cpu().numpy(), O.unpack_nibbles(wp.numpy()))
+
+
 # ------------------------------------------------------- integer GEMM (exact)
 
 GEMM_SHAPES = [(128, 128, 256), (300, 384, 520), (1, 32, 8), (257, 4096, 300), (129, 160, 257),
@@ -144,6 +168,16 @@ def test_gemm_w4a8_i32_bit_exact(ck, M, K, N):
     wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
     acc = ck.gemm_w4a8_i32(qa.to(DEV), wp.to(DEV))
     ref = O.int_matmul(qa.numpy().astype(np.int64), O.unpack_nibbles(wp.numpy()))
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("M,K,N", GEMM_SHAPES)
+def test_gemm_s8_i32_bit_exact(ck, M, K, N):
+    g = torch.Generator().manual_seed(M * 13 + N)
+    qa = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    w8 = torch.randint(-128, 128, (N, K), generator=g, dtype=torch.int8)
+    acc = ck.gemm_s8_i32(qa.to(DEV), w8.to(DEV))
+    ref = O.int_matmul(qa.numpy().astype(np.int64), w8.numpy().astype(np.int64))
     np.testing.assert_array_equal(acc.cpu().numpy(), ref)
 
 
@@ -174,6 +208,23 @@ def test_gemm_w4a4_epilogue_bit_exact(ck, M, K, N, with_bias):
     np.testing.assert_array_equal(bf16_tensor_bits(y), ref_bits)
 
 
+@pytest.mark.parametrize("M,K,N", [(200, 512, 300), (8192, 3840, 256), (45, 160, 70)])
+def test_gemm_w4a8_and_s8_epilogue_bit_exact(ck, M, K, N):
+    g = torch.Generator().manual_seed(M * 3 + N)
+    qa = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    sa = torch.rand(M, generator=g) * 0.5 + 0.01
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N,), 0.005, 0.02, g)
+    bias = WL.uniform((N,), -1, 1, g)
+    acc = O.int_matmul(qa.numpy().astype(np.int64), O.unpack_nibbles(wp.numpy()))
+    ref_bits = O.to_bf16_bits(O.epilogue_rowwise(acc, sa.numpy(), to_np_f64(sw), to_np_f64(bias)))
+    y = ck.gemm_w4a8(qa.to(DEV), sa.to(DEV), wp.to(DEV), sw.to(DEV), bias.to(DEV))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), ref_bits)
+    w8 = ck.unpack_int4(wp.to(DEV))
+    y8 = ck.gemm_s8(qa.to(DEV), sa.to(DEV), w8, sw.to(DEV), bias.to(DEV))
+    np.testing.assert_array_equal(bf16_tensor_bits(y8), ref_bits)
+
+
 # --------------------------------------------------------- W4A4 linear (e2e)
 
 @pytest.mark.parametrize("M,K,N,G,bias,dtype", [
@@ -200,16 +251,17 @@ def _linear_full_config(ck, w, sample_rows):
     torch.cuda.synchronize()
     rows = np.asarray(sample_rows)
     r = O.linear_w4a4(to_np_f64(d["x"][rows]), d["w_packed"].numpy(), to_np_f64(d["w_scale"]), w.G)
-    # the quantized activations the GEMM consumed (workspace: packed codes, then scales)
-    nq = w.M * (w.K // 2)
-    qa = ws[:nq].view(w.M, w.K // 2).cpu()[rows]
+    # the quantized activations the GEMM consumed (workspace: int8 codes, then scales)
+    nq = w.M * w.K
+    qa = ws[:nq].view(torch.int8).view(w.M, w.K).cpu().numpy()[rows].astype(np.int64)
     off = (nq + 255) // 256 * 256
     sa = ws[off:off + 4 * w.M].view(torch.float32).cpu().numpy()[rows]
-    assert_codes_close(unpack_codes(qa), r["q"])
+    assert qa.min() >= -7 and qa.max() <= 7
+    assert_codes_close(qa, r["q"])
     assert_scales_close(sa, r["s"])
     rel = assert_out_close(to_np_f64(y.cpu()[rows]), O.bf16_bits_to_f64(r["y_bits"]))
     # with identical quantized inputs the GEMM + epilogue is bit-exact
-    acc = O.int_matmul(unpack_codes(qa), O.unpack_nibbles(d["w_packed"].numpy()))
+    acc = O.int_matmul(qa, O.unpack_nibbles(d["w_packed"].numpy()))
     exact = O.to_bf16_bits(O.epilogue_rowwise(acc, sa, to_np_f64(d["w_scale"])))
     np.testing.assert_array_equal(bf16_tensor_bits(y.cpu()[rows]), exact)
     return rel
