@@ -9,7 +9,7 @@ ImportError if it has not been built (there is no CPU fallback).
 _OPS = ("rotate_quant_rowwise", "gemm_w4a4", "linear_w4a4", "linear_w4a4_workspace_bytes",
         "gemv_w4a8", "gemv_awq_w4a16", "gemm_w4a4_i32", "gemm_w4a8_i32", "device_error_check",
         "selftest_bounded_wait", "CKError", "version", "rotate_quant_rowwise_i8", "unpack_int4",
-        "gemm_s8", "gemm_s8_i32", "gemm_w4a8")
+        "gemm_s8", "gemm_s8_i32", "gemm_w4a8", "linear_w4a4_quantize", "linear_w4a4_matmul")
 
 __all__ = list(_OPS) + ["ck", "workloads"]
 

@@ -44,6 +44,8 @@ SIGNATURES = {
     "ck_gemm_s8_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
     "ck_linear_w4a4_workspace_bytes": [_i64, _i64],
     "ck_linear_w4a4": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
+    "ck_linear_w4a4_quantize": [_p, _int, _i64, _i64, _i64, _int, _p, ctypes.c_size_t, _p],
+    "ck_linear_w4a4_matmul": [_i64, _i64, _i64, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
     "ck_gemv_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemv_awq_w4a16": [_p, _int, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p],
     "ck_gemm_w4a4_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
@@ -223,6 +225,28 @@ def linear_w4a4(x, w_packed, w_scale, group_size: int, bias=None, workspace=None
                               _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)),
            "ck_linear_w4a4")
+    return out
+
+
+def linear_w4a4_quantize(x, group_size: int, workspace, stream=None):
+    """Phase 1 of linear_w4a4: rotate + quantize x into `workspace` (opaque)."""
+    _cuda(x, workspace)
+    M, K, ldx, x2 = _rows(x)
+    _check(lib.ck_linear_w4a4_quantize(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)),
+           "ck_linear_w4a4_quantize")
+    return workspace
+
+
+def linear_w4a4_matmul(M: int, K: int, w_packed, w_scale, workspace, bias=None, out=None, stream=None):
+    """Phase 2 of linear_w4a4: GEMM of the workspace codes with the packed weights -> y (M, N) bf16."""
+    _cuda(w_packed, w_scale, workspace, bias)
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=w_packed.device, dtype=torch.bfloat16)
+    _check(lib.ck_linear_w4a4_matmul(M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias), _ptr(out),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "ck_linear_w4a4_matmul")
     return out
 
 

@@ -102,31 +102,32 @@ ck_status ensure_smem_attr(KernelT kernel, size_t bytes) {
 }
 
 template <int QBITS, int STORE, typename T>
-void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s, int nt,
+void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s, int32_t* rs, int nt,
                cudaStream_t st) {
   const float rnorm = (float)(1.0 / std::sqrt((double)G));
   ck::rq::rotate_quant_kernel<QBITS, STORE, T><<<(unsigned)M, nt, 0, st>>>(
-      reinterpret_cast<const T*>(x), K, ldx, G, rnorm, reinterpret_cast<uint8_t*>(q), s);
+      reinterpret_cast<const T*>(x), K, ldx, G, rnorm, reinterpret_cast<uint8_t*>(q), s, rs);
 }
 
-// store: ck::rq::STORE_PACKED4 (bits must be 4) or ck::rq::STORE_INT8 (codes as int8 bytes).
+template <typename T>
+void launch_rq_store(int bits, int store, const void* x, int64_t M, int K, int64_t ldx, int G, void* q,
+                     float* s, int32_t* rs, int nt, cudaStream_t st) {
+  using namespace ck::rq;
+  if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, K, ldx, G, q, s, rs, nt, st);
+  else if (store == STORE_INT8_PERM) launch_rq<4, STORE_INT8_PERM, T>(x, M, K, ldx, G, q, s, rs, nt, st);
+  else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, st);
+  else launch_rq<8, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, st);
+}
+
+// store: STORE_PACKED4 (bits 4), STORE_INT8 (codes as int8 bytes) or STORE_INT8_PERM
+// (bits 4, the linear's GEMM-ready activations with row sums in `rs`).
 ck_status rotate_quant_impl(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int G,
-                            int bits, int store, void* q, float* s, cudaStream_t st) {
+                            int bits, int store, void* q, float* s, int32_t* rs, cudaStream_t st) {
   using namespace ck::rq;
   const int64_t nt = ((K + EPT - 1) / EPT + 31) / 32 * 32;
   if (nt > 1024) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K=%lld too large (max 32768)", (long long)K);
-  const int k = (int)K, n = (int)nt;
-  if (xt == CK_BF16) {
-    using T = __nv_bfloat16;
-    if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, k, ldx, G, q, s, n, st);
-    else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
-    else launch_rq<8, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
-  } else {
-    using T = __half;
-    if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, k, ldx, G, q, s, n, st);
-    else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
-    else launch_rq<8, STORE_INT8, T>(x, M, k, ldx, G, q, s, n, st);
-  }
+  if (xt == CK_BF16) launch_rq_store<__nv_bfloat16>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, st);
+  else launch_rq_store<__half>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, st);
   return launch_status("rotate_quant");
 }
 
@@ -140,9 +141,36 @@ ck_status check_gemm_shape(const char* who, int64_t M, int64_t K, int64_t N) {
   return CK_OK;
 }
 
+// Largest number of CTA pairs of this kernel that are co-resident on the device (cached per device).
+template <typename Tag, typename KernelT>
+ck_status max_pairs(KernelT kernel, size_t smem, int* out) {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(CK_ERR_CUDA, "cudaGetDevice failed");
+  if (cache[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(ck::gemm::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+    if (e != cudaSuccess || n <= 0) return fail(CK_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s (%d)", cudaGetErrorString(e), n);
+    cache[dev] = n;
+  }
+  *out = cache[dev];
+  return CK_OK;
+}
+
 template <int A_MODE, int B_MODE, int EPI>
-ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const void* w,
-                    const float* a_scale, const uint16_t* w_scale, const uint16_t* bias, void* out,
+ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const void* w, const float* a_scale,
+                    const int32_t* a_rowsum, const uint16_t* w_scale, const uint16_t* bias, void* out,
                     cudaStream_t st) {
   using namespace ck::gemm;
   using C = Cfg<A_MODE, B_MODE>;
@@ -151,26 +179,75 @@ ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const void*
   if (C::AP) r = make_tmap(&ta, qa, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, PKB, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
   else r = make_tmap(&ta, qa, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (r != CK_OK) return r;
-  if (C::BP) r = make_tmap(&tb, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, PKB, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
-  else r = make_tmap(&tb, w, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (C::BP) r = make_tmap(&tb, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, PKB, BNH, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else r = make_tmap(&tb, w, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BNH, CU_TENSOR_MAP_SWIZZLE_128B);
   if (r != CK_OK) return r;
   auto kern = gemm_w4_kernel<A_MODE, B_MODE, EPI>;
   struct Tag {};
   if ((r = ensure_smem_attr<Tag>(kern, C::SMEM)) != CK_OK) return r;
+  int pairs_max = 0;
+  if ((r = max_pairs<Tag>(kern, C::SMEM, &pairs_max)) != CK_OK) return r;
   Params p;
   p.M = (int)M; p.N = (int)N; p.K = (int)K;
+  p.tiles_m = (int)((M + 2 * BM - 1) / (2 * BM));
+  p.tiles_n = (int)((N + BN - 1) / BN);
   p.a_scale = a_scale;
+  p.a_rowsum = a_rowsum;
   p.w_scale = reinterpret_cast<const __nv_bfloat16*>(w_scale);
   p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
   p.out = out;
   const size_t esz = EPI == EPI_I32 ? 4 : 2;
   p.out_vec_ok = aligned(out, 16) && ((N * (int64_t)esz) % 16 == 0);
-  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-  kern<<<grid, kThreads, C::SMEM, st>>>(ta, tb, p);
+  const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
+  const int pairs = (int)std::min<int64_t>(tiles, pairs_max);
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemm_w4: launch failed: %s", cudaGetErrorString(e));
   return launch_status("gemm_w4");
 }
 
-size_t linear_q_bytes(int64_t M, int64_t K) { return ((size_t)M * (size_t)K + 255) / 256 * 256; }
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+size_t linear_q_bytes(int64_t M, int64_t K) { return align256((size_t)M * (size_t)K); }
+
+// The linear's workspace: int8 codes (M, K) in the GEMM's permuted column order,
+// float32 row scales (M), int32 row sums of the codes (M), each 256-byte aligned.
+struct LinearWs {
+  int8_t* q;
+  float* scale;
+  int32_t* rowsum;
+};
+
+LinearWs linear_ws(void* base, int64_t M, int64_t K) {
+  uint8_t* b = reinterpret_cast<uint8_t*>(base);
+  LinearWs w;
+  w.q = reinterpret_cast<int8_t*>(b);
+  w.scale = reinterpret_cast<float*>(b + linear_q_bytes(M, K));
+  w.rowsum = reinterpret_cast<int32_t*>(b + linear_q_bytes(M, K) + align256((size_t)M * sizeof(float)));
+  return w;
+}
+
+size_t linear_ws_bytes(int64_t M, int64_t K) {
+  return linear_q_bytes(M, K) + align256((size_t)M * sizeof(float)) + (size_t)M * sizeof(int32_t);
+}
+
+ck_status check_linear_workspace(const char* who, int64_t M, int64_t K, const void* ws, size_t bytes) {
+  if (ws == nullptr || bytes < linear_ws_bytes(M, K))
+    return fail(CK_ERR_INVALID_ARG, "%s: workspace smaller than ck_linear_w4a4_workspace_bytes", who);
+  if (!aligned(ws, 256)) return fail(CK_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  return CK_OK;
+}
 
 }  // namespace
 
@@ -199,7 +276,7 @@ ck_status ck_rotate_quant_rowwise(const void* x, ck_dtype xt, int64_t M, int64_t
   if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: M too large");
   return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits,
                            bits == 4 ? ck::rq::STORE_PACKED4 : ck::rq::STORE_INT8, q_out, scale_out,
-                           S(stream));
+                           nullptr, S(stream));
 }
 
 ck_status ck_rotate_quant_rowwise_i8(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
@@ -219,7 +296,8 @@ ck_status ck_rotate_quant_rowwise_i8(const void* x, ck_dtype xt, int64_t M, int6
   if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: x rows must be 16-byte aligned");
   if (!aligned(q_out, 16) || !aligned(scale_out, 4)) return fail(CK_ERR_INVALID_ARG, "rotate_quant_i8: misaligned output");
   if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "rotate_quant_i8: M too large");
-  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, ck::rq::STORE_INT8, q_out, scale_out, S(stream));
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, ck::rq::STORE_INT8, q_out, scale_out, nullptr,
+                           S(stream));
 }
 
 ck_status ck_unpack_int4(const uint8_t* packed, int64_t R, int64_t C, int8_t* out, void* stream) {
@@ -244,7 +322,7 @@ ck_status ck_gemm_s8(const int8_t* qa, const float* a_scale, int64_t M, int64_t 
   if (!aligned(qa, 16) || !aligned(w, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_s8: operands must be 16-byte aligned");
   if (!aligned(a_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "gemm_s8: misaligned scale, bias or output");
-  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_BF16>(qa, M, K, N, w, a_scale, w_scale, bias, y, S(stream));
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_BF16>(qa, M, K, N, w, a_scale, nullptr, w_scale, bias, y, S(stream));
 }
 
 ck_status ck_gemm_w4a8(const int8_t* qa, const float* a_scale, int64_t M, int64_t K, int64_t N,
@@ -256,7 +334,7 @@ ck_status ck_gemm_w4a8(const int8_t* qa, const float* a_scale, int64_t M, int64_
   if (!aligned(qa, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a8: operands must be 16-byte aligned");
   if (!aligned(a_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "gemm_w4a8: misaligned scale, bias or output");
-  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4, ck::gemm::EPI_BF16>(qa, M, K, N, w_packed, a_scale, w_scale, bias, y, S(stream));
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4, ck::gemm::EPI_BF16>(qa, M, K, N, w_packed, a_scale, nullptr, w_scale, bias, y, S(stream));
 }
 
 ck_status ck_gemm_s8_i32(const int8_t* qa, const int8_t* w, int64_t M, int64_t K, int64_t N, int32_t* acc,
@@ -266,7 +344,7 @@ ck_status ck_gemm_s8_i32(const int8_t* qa, const int8_t* w, int64_t M, int64_t K
   if (!qa || !w || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_s8_i32: null pointer");
   if (!aligned(qa, 16) || !aligned(w, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_s8_i32: operands must be 16-byte aligned");
   if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_s8_i32: misaligned output");
-  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_I32>(qa, M, K, N, w, nullptr, nullptr, nullptr, acc, S(stream));
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_I32>(qa, M, K, N, w, nullptr, nullptr, nullptr, nullptr, acc, S(stream));
 }
 
 ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M, int64_t K,
@@ -278,12 +356,44 @@ ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M
   if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4: operands must be 16-byte aligned");
   if (!aligned(a_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "gemm_w4a4: misaligned scale, bias or output");
-  return gemm_impl<ck::gemm::OP_PACKED4, ck::gemm::OP_PACKED4, ck::gemm::EPI_BF16>(qa_packed, M, K, N, w_packed, a_scale, w_scale, bias, y, S(stream));
+  return gemm_impl<ck::gemm::OP_PACKED4, ck::gemm::OP_PACKED4, ck::gemm::EPI_BF16>(qa_packed, M, K, N, w_packed, a_scale, nullptr, w_scale, bias, y, S(stream));
 }
 
 size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K) {
   if (M <= 0 || K <= 0) return 0;
-  return linear_q_bytes(M, K) + (size_t)M * sizeof(float);
+  return linear_q_bytes(M, K) + align256((size_t)M * sizeof(float)) + (size_t)M * sizeof(int32_t);
+}
+
+ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int group_size,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  ck_status r = check_gemm_shape("linear_w4a4_quantize", M, K, 1);
+  if (r != CK_OK) return r;
+  if ((r = check_linear_workspace("linear_w4a4_quantize", M, K, workspace, ws_bytes)) != CK_OK) return r;
+  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: unknown dtype");
+  if (!is_pow2(group_size) || group_size > 256)
+    return fail(CK_ERR_UNSUPPORTED, "linear_w4a4_quantize: group_size=%d must be a power of two <= 256", group_size);
+  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: K %% group_size != 0");
+  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: ldx < K");
+  if (x == nullptr) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: null pointer");
+  if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: x rows must be 16-byte aligned");
+  LinearWs ws = linear_ws(workspace, M, K);
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, 4, ck::rq::STORE_INT8_PERM, ws.q, ws.scale, ws.rowsum,
+                           S(stream));
+}
+
+ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
+                                const uint16_t* bias, uint16_t* y, const void* workspace, size_t ws_bytes,
+                                void* stream) {
+  ck_status r = check_gemm_shape("linear_w4a4_matmul", M, K, N);
+  if (r != CK_OK) return r;
+  if ((r = check_linear_workspace("linear_w4a4_matmul", M, K, workspace, ws_bytes)) != CK_OK) return r;
+  if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_matmul: null pointer");
+  if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "linear_w4a4_matmul: weights must be 16-byte aligned");
+  if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "linear_w4a4_matmul: misaligned scale, bias or output");
+  LinearWs ws = linear_ws(const_cast<void*>(workspace), M, K);
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4_U, ck::gemm::EPI_BF16>(
+      ws.q, M, K, N, w_packed, ws.scale, ws.rowsum, w_scale, bias, y, S(stream));
 }
 
 ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
@@ -292,19 +402,15 @@ ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64
                          void* stream) {
   ck_status r = check_gemm_shape("linear_w4a4", M, K, N);
   if (r != CK_OK) return r;
-  if (!workspace || ws_bytes < ck_linear_w4a4_workspace_bytes(M, K))
-    return fail(CK_ERR_INVALID_ARG, "linear_w4a4: workspace smaller than ck_linear_w4a4_workspace_bytes");
-  if (!aligned(workspace, 256)) return fail(CK_ERR_INVALID_ARG, "linear_w4a4: workspace must be 256-byte aligned");
+  // validate both phases before enqueuing either
+  if ((r = check_linear_workspace("linear_w4a4", M, K, workspace, ws_bytes)) != CK_OK) return r;
   if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "linear_w4a4: null pointer");
   if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "linear_w4a4: weights must be 16-byte aligned");
   if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "linear_w4a4: misaligned scale, bias or output");
-  // int4 codes (|q| <= 7) stored one per byte: the GEMM reads them with TMA, no activation unpack
-  int8_t* qa = reinterpret_cast<int8_t*>(workspace);
-  float* sa = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + linear_q_bytes(M, K));
-  r = ck_rotate_quant_rowwise_i8(x, xt, M, K, ldx, group_size, 4, qa, sa, stream);
+  r = ck_linear_w4a4_quantize(x, xt, M, K, ldx, group_size, workspace, ws_bytes, stream);
   if (r != CK_OK) return r;
-  return ck_gemm_w4a8(qa, sa, M, K, N, w_packed, w_scale, bias, y, stream);
+  return ck_linear_w4a4_matmul(M, K, N, w_packed, w_scale, bias, y, workspace, ws_bytes, stream);
 }
 
 ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, int64_t M, int64_t K,
@@ -314,7 +420,7 @@ ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, in
   if (!qa_packed || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4_i32: null pointer");
   if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4_i32: operands must be 16-byte aligned");
   if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4_i32: misaligned output");
-  return gemm_impl<ck::gemm::OP_PACKED4, ck::gemm::OP_PACKED4, ck::gemm::EPI_I32>(qa_packed, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
+  return gemm_impl<ck::gemm::OP_PACKED4, ck::gemm::OP_PACKED4, ck::gemm::EPI_I32>(qa_packed, M, K, N, w_packed, nullptr, nullptr, nullptr, nullptr, acc, S(stream));
 }
 
 ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M, int64_t K, int64_t N,
@@ -324,7 +430,7 @@ ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M,
   if (!qa || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8_i32: null pointer");
   if (!aligned(qa, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a8_i32: operands must be 16-byte aligned");
   if (!aligned(acc, 4)) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8_i32: misaligned output");
-  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4, ck::gemm::EPI_I32>(qa, M, K, N, w_packed, nullptr, nullptr, nullptr, acc, S(stream));
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4, ck::gemm::EPI_I32>(qa, M, K, N, w_packed, nullptr, nullptr, nullptr, nullptr, acc, S(stream));
 }
 
 ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,

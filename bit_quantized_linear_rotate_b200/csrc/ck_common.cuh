@@ -89,6 +89,67 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Cluster-scope variants, for barriers that receive arrivals from the peer CTA
+// of a CTA pair (and whose waiters read data that CTA produced).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                  unsigned int site, uint64_t limit_ns = kDefaultWaitNs) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 255u) == 0u) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (abort != nullptr) *abort = 1;
+        report_timeout(site);
+        return false;
+      }
+    }
+  }
+}
+
+// Every lane of the warp waits (bounded); the warp proceeds only if all lanes saw the phase.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned int site) {
+  const bool ok = mbar_wait(bar, parity, abort, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// ------------------------------------------------------------------ cluster
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+
+// Arrive (release at cluster scope) on a barrier given by its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // --------------------------------------------------------------------- TMA
 
 // 2-D tiled TMA load (no multicast): box at coordinates (x = inner, y = row).
@@ -98,6 +159,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
       "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Tile load by either CTA of a pair, completing bytes on the barrier at the
+// shared::cluster address `bar_cluster` (the leader CTA's). No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tmap, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
 }
 
@@ -156,6 +228,44 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// ---- CTA-pair (cta_group::2) forms: issued by the leader CTA, operands and
+// accumulator split across the pair by M, the B operand split by N.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives on the barrier at this offset in every CTA of `cta_mask` once the
+// pair's tcgen05 operations issued so far by this thread have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane
 // (base lane + i), columns [col, col + 32).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -188,11 +298,11 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(const void* tile, uint32_t
   return lo | (hi << 32);
 }
 
-// Instruction descriptor for kind::i8: signed A and B, int32 accumulator,
-// both operands K-major, tile M x N.
-__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(N) >> 3) << 17) |
-         ((uint32_t(M) >> 4) << 24);
+// Instruction descriptor for kind::i8: int32 accumulator, both operands
+// K-major, tile M x N; A and B signed (1) or unsigned (0).
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool a_signed = true, bool b_signed = true) {
+  return (2u << 4) | ((a_signed ? 1u : 0u) << 7) | ((b_signed ? 1u : 0u) << 10) |
+         ((uint32_t(N) >> 3) << 17) | ((uint32_t(M) >> 4) << 24);
 }
 
 // ------------------------------------------------------------ packed nibbles
@@ -217,6 +327,14 @@ __device__ __forceinline__ void decode_nibbles_s8(const uint4 p, uint4& o0, uint
   }
   o0 = make_uint4(r[0], r[1], r[2], r[3]);
   o1 = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+// 16 packed bytes -> 32 unsigned nibbles u in [0, 15] with the k order of each
+// 8-column group permuted to (0 2 4 6 1 3 5 7): the low nibbles of a word, then
+// its high nibbles. Pairs with activations stored in the same permuted order.
+__device__ __forceinline__ void decode_nibbles_u8_perm(const uint4 p, uint4& o0, uint4& o1) {
+  o0 = make_uint4(p.x & 0x0F0F0F0Fu, (p.x >> 4) & 0x0F0F0F0Fu, p.y & 0x0F0F0F0Fu, (p.y >> 4) & 0x0F0F0F0Fu);
+  o1 = make_uint4(p.z & 0x0F0F0F0Fu, (p.z >> 4) & 0x0F0F0F0Fu, p.w & 0x0F0F0F0Fu, (p.w >> 4) & 0x0F0F0F0Fu);
 }
 
 }  // namespace ck

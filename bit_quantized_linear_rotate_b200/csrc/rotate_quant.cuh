@@ -14,9 +14,12 @@
 // never leaves registers: amax is reduced across the CTA, then every thread
 // quantizes its 32 values and writes 16 bytes (packed int4) or 32 bytes (int8).
 //
-// Quantization multiplies by the reciprocal of the scale; when the product lies
-// within 1e-4 of a rounding boundary it is recomputed with the correctly
-// rounded quotient y / s, so ties are decided as by division.
+// Arithmetic is packed two lanes at a time (sm_100 f32x2 add/mul/fma). Codes
+// are rounded by adding 1.5 * 2^23 (round to nearest, ties to even, no float to
+// int conversion) and packed with byte permutes. Quantization multiplies by
+// the reciprocal of the scale; for unrotated rows (G = 1, where exact halves
+// are common) codes near a half integer are decided exactly by the sign of
+// y - h s, as division would.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -29,7 +32,11 @@ namespace rq {
 
 constexpr int EPT = 32;   // columns per thread
 
-enum Store { STORE_PACKED4 = 0, STORE_INT8 = 1 };
+// STORE_INT8_PERM: int8 codes with the columns of each 8-column group stored in
+// the order (0 2 4 6 1 3 5 7), plus the row sum of the codes -- the activation
+// format of the linear's GEMM (it pairs with weights split into low / high
+// nibbles without byte shuffles).
+enum Store { STORE_PACKED4 = 0, STORE_INT8 = 1, STORE_INT8_PERM = 2 };
 
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float* f);
@@ -57,18 +64,31 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float* f) {
   }
 }
 
+// The 32 values of a thread live as 16 float2 pairs v[j] = (y[2j], y[2j+1]);
+// sm_100 executes one f32x2 add / fma per pair, two lanes of fp32 work.
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {       // a - b, one rounding
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
 // Sylvester butterflies on element-index bits below min(G, 32): for index bit h,
 // (a, b) -> (a + b, a - b) where a has the bit clear.
-__device__ __forceinline__ void fht_in_thread(float (&v)[EPT], int G) {
+__device__ __forceinline__ void fht_in_thread(float2 (&v)[EPT / 2], int G) {
+  if (G > 1) {
 #pragma unroll
-  for (int h = 1; h < EPT; h <<= 1) {
-    if (h < G) {
+    for (int j = 0; j < EPT / 2; ++j) {
+      const float a = v[j].x, b = v[j].y;
+      v[j] = make_float2(a + b, a - b);
+    }
+  }
 #pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        if ((e & h) == 0) {
-          const float a = v[e], b = v[e + h];
-          v[e] = a + b;
-          v[e + h] = a - b;
+  for (int hb = 1; hb < EPT / 2; hb <<= 1) {       // element bit 1.. = pair-index bit 0..
+    if (2 * hb < G) {
+#pragma unroll
+      for (int j = 0; j < EPT / 2; ++j) {
+        if ((j & hb) == 0) {
+          const float2 a = v[j], b = v[j + hb];
+          v[j] = __fadd2_rn(a, b);
+          v[j + hb] = sub2(a, b);
         }
       }
     }
@@ -76,28 +96,41 @@ __device__ __forceinline__ void fht_in_thread(float (&v)[EPT], int G) {
 }
 
 // Index bits 5.. live in lane bits 0..: new = partner + v (bit clear) or partner - v (bit set).
-__device__ __forceinline__ void fht_across_lanes(float (&v)[EPT], int G, int lane) {
+__device__ __forceinline__ void fht_across_lanes(float2 (&v)[EPT / 2], int G, int lane) {
   for (int j = 1; EPT * j < G; j <<= 1) {
-    const float sgn = (lane & j) ? -1.0f : 1.0f;
+    const float sg = (lane & j) ? -1.0f : 1.0f;
+    const float2 sgn = make_float2(sg, sg);
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-      const float other = __shfl_xor_sync(0xffffffffu, v[e], j);
-      v[e] = fmaf(sgn, v[e], other);
+    for (int e = 0; e < EPT / 2; ++e) {
+      const float2 other = make_float2(__shfl_xor_sync(0xffffffffu, v[e].x, j),
+                                       __shfl_xor_sync(0xffffffffu, v[e].y, j));
+      v[e] = __ffma2_rn(sgn, v[e], other);
     }
   }
 }
 
-__device__ __forceinline__ int quant1(float y, float r, float s, float qmax) {
-  float t = __fmul_rn(y, r);
-  const float f = t - truncf(t);
-  if (fabsf(fabsf(f) - 0.5f) < 1e-4f) t = __fdiv_rn(y, s);
-  return (int)fminf(fmaxf(rintf(t), -qmax), qmax);
+// Adding 1.5 * 2^23 rounds |t| < 2^22 to an integer (nearest, ties to even) in
+// the low mantissa bits: the float's bit pattern is 0x4B400000 + round(t).
+constexpr float kRoundMagic = 12582912.0f;
+
+// Exact round-half-even of y / s for an unrotated row (y = x exactly): the
+// reciprocal product decides every code that is not within 1e-3 of a half
+// integer; near one, the sign of the single-rounding residual y - h s decides.
+__device__ __forceinline__ float quant_exact(float y, float r, float s) {
+  const float t = __fmul_rn(y, r);
+  const float fl = floorf(t);
+  const float d = t - fl;
+  if (fabsf(d - 0.5f) >= 1e-3f) return rintf(t);
+  const float h = fl + 0.5f;
+  const float e = fmaf(-h, s, y);
+  return e > 0.0f ? fl + 1.0f : (e < 0.0f ? fl : rintf(h));
 }
 
 template <int QBITS, int STORE, typename T>
 __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict__ x, int K, int64_t ldx,
                                                             int G, float rnorm, uint8_t* __restrict__ q,
-                                                            float* __restrict__ scale) {
+                                                            float* __restrict__ scale,
+                                                            int32_t* __restrict__ rowsum) {
   constexpr float kQmax = QBITS == 4 ? 7.0f : 127.0f;
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
@@ -106,26 +139,26 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
   const int e0 = tid * EPT;
   const T* xr = x + row * ldx;
 
-  float v[EPT];
+  float2 v[EPT / 2];
 #pragma unroll
   for (int j = 0; j < EPT / 8; ++j) {
+    float f[8];
     if (e0 + 8 * j < K) {
-      load8<T>(xr + e0 + 8 * j, v + 8 * j);
+      load8<T>(xr + e0 + 8 * j, f);
     } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[8 * j + e] = 0.0f;
+      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[4 * j + e] = make_float2(f[2 * e], f[2 * e + 1]);
   }
 
-  if (G > 1) {
-    fht_in_thread(v, G);
-    fht_across_lanes(v, G, lane);   // every lane runs it; columns past K hold zeros
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) v[e] *= rnorm;
-  }
+  // unnormalised transform z = x H; the 1/sqrt(G) factor is folded into the scale
+  fht_in_thread(v, G);
+  if (G > EPT) fht_across_lanes(v, G, lane);   // every lane runs it; columns past K hold zeros
   float amax = 0.0f;
 #pragma unroll
-  for (int e = 0; e < EPT; ++e) amax = fmaxf(amax, fabsf(v[e]));
+  for (int e = 0; e < EPT / 2; ++e) amax = fmaxf(amax, fmaxf(fabsf(v[e].x), fabsf(v[e].y)));
 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -138,23 +171,66 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
     if (tid == 0) red[0] = a;
   }
   __syncthreads();
-  amax = red[0];
+  amax = __fmul_rn(red[0], rnorm);               // amax of y = z / sqrt(G)
 
   // positive-scale contract: an all-zero row gets scale 1 and all-zero codes
   const float s = amax > 0.0f ? __fdiv_rn(amax, kQmax) : 1.0f;
   const float r = __frcp_rn(s);
   if (tid == 0) scale[row] = s;
+
+  // codes: bit patterns whose low byte is q (int8) or q + 8 (offset-binary int4)
+  uint32_t u[EPT];
+  const float magic = STORE == STORE_PACKED4 ? kRoundMagic + 8.0f : kRoundMagic;
+  if (G == 1) {
+#pragma unroll
+    for (int e = 0; e < EPT / 2; ++e) {
+      u[2 * e] = __float_as_uint(quant_exact(v[e].x, r, s) + magic);
+      u[2 * e + 1] = __float_as_uint(quant_exact(v[e].y, r, s) + magic);
+    }
+  } else {
+    const float rr = __fmul_rn(r, rnorm);          // exact for G = 4^k (rnorm a power of two)
+    const float2 r2 = make_float2(rr, rr), m2 = make_float2(magic, magic);
+#pragma unroll
+    for (int e = 0; e < EPT / 2; ++e) {
+      const float2 t = __fadd2_rn(__fmul2_rn(v[e], r2), m2);
+      u[2 * e] = __float_as_uint(t.x);
+      u[2 * e + 1] = __float_as_uint(t.y);
+    }
+  }
+  // low bytes of four codes -> one word (natural order, or (0 2 4 6)(1 3 5 7) per 8 columns)
+  uint32_t g[EPT / 4];
+#pragma unroll
+  for (int j = 0; j < EPT / 4; ++j) {
+    const int b = STORE == STORE_INT8_PERM ? 8 * (j >> 1) + (j & 1) : 4 * j;
+    const int st = STORE == STORE_INT8_PERM ? 2 : 1;
+    g[j] = __byte_perm(__byte_perm(u[b], u[b + st], 0x5140), __byte_perm(u[b + 2 * st], u[b + 3 * st], 0x5140),
+                       0x5410);
+  }
+  if (STORE == STORE_INT8_PERM) {
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < EPT / 4; ++j) sum = __dp4a((int)g[j], 0x01010101, sum);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    __syncthreads();                                  // red[] is free again
+    if (lane == 0) red[tid >> 5] = __int_as_float(sum);
+    __syncthreads();
+    if (tid < 32) {
+      int a = tid < (int)(blockDim.x >> 5) ? __float_as_int(red[tid]) : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (tid == 0) rowsum[row] = a;
+    }
+  }
   if (e0 >= K) return;
 
   if (STORE == STORE_PACKED4) {
-    // 32 codes -> 16 bytes, u = q + 8, low nibble = even column
+    // bytes hold u = q + 8 < 16: fold neighbours into nibbles, low nibble = even column
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      uint32_t acc = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc |= (uint32_t)(quant1(v[8 * j + e], r, s, kQmax) + 8) << (4 * e);
-      w[j] = acc;
+      const uint32_t ta = g[2 * j] | (g[2 * j] >> 4), tb = g[2 * j + 1] | (g[2 * j + 1] >> 4);
+      w[j] = __byte_perm(ta, tb, 0x6420);
     }
     uint8_t* qr = q + row * (int64_t)(K >> 1) + (e0 >> 1);
     if ((K & 31) == 0) {          // rows of K/2 bytes are 16-byte aligned
@@ -165,22 +241,14 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
         if (e0 + 8 * j < K) reinterpret_cast<uint32_t*>(qr)[j] = w[j];
     }
   } else {
-    uint32_t w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint32_t acc = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc |= (uint32_t)(quant1(v[4 * j + e], r, s, kQmax) & 0xFF) << (8 * e);
-      w[j] = acc;
-    }
     uint8_t* qr = q + row * (int64_t)K + e0;
     if ((K & 31) == 0) {
-      reinterpret_cast<uint4*>(qr)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      reinterpret_cast<uint4*>(qr)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      reinterpret_cast<uint4*>(qr)[0] = make_uint4(g[0], g[1], g[2], g[3]);
+      reinterpret_cast<uint4*>(qr)[1] = make_uint4(g[4], g[5], g[6], g[7]);
     } else {
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (e0 + 8 * j < K) reinterpret_cast<uint2*>(qr)[j] = make_uint2(w[2 * j], w[2 * j + 1]);
+        if (e0 + 8 * j < K) reinterpret_cast<uint2*>(qr)[j] = make_uint2(g[2 * j], g[2 * j + 1]);
     }
   }
 }

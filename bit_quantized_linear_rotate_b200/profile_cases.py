@@ -9,6 +9,8 @@ Cases (full workload sizes, a few GB at most on the device):
   gemm_s8_M8192    ck_gemm_s8 with pre-decoded int8 weights
   gemm_w4a4_M8192  ck_gemm_w4a4, packed int4 activations and weights
   linear_M8192     ck_linear_w4a4 (both kernels)
+  linmm_M8192      ck_linear_w4a4_matmul (the linear's GEMM phase alone)
+  linq_M8192       ck_linear_w4a4_quantize (the linear's rotate + quantize phase alone)
   w4a8_M{1,4,16}   ck_gemv_w4a8, K=4096, N=12288
   awq_M{1,2,4}     ck_gemv_awq_w4a16, K=3072, N=18432, G=64
 One warm-up call precedes the timed iterations; the process exits non-zero if
@@ -45,9 +47,14 @@ def build_case(name: str, dev):
         if name == "gemm_w4a4_M8192":
             qp, _ = ck.rotate_quant_rowwise(x, w.G, 4)
             return lambda: ck.gemm_w4a4(qp, sa, wp, sw, out=y)
+        ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
         if name == "linear_M8192":
-            ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
             return lambda: ck.linear_w4a4(x, wp, sw, w.G, workspace=ws, out=y)
+        if name == "linq_M8192":
+            return lambda: ck.linear_w4a4_quantize(x, w.G, ws)
+        if name == "linmm_M8192":
+            ck.linear_w4a4_quantize(x, w.G, ws)
+            return lambda: ck.linear_w4a4_matmul(w.M, w.K, wp, sw, ws, out=y)
     if name.startswith("w4a8_M"):
         M = int(name[len("w4a8_M"):])
         d = WL.gemv_w4a8_inputs(WL.GEMV_W4A8, M)

@@ -137,18 +137,35 @@ size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K);
 /*
  * The ConvRot W4A4 linear ("public ConvRot W4A4 Linear dispatcher",
  * comfy-kitchen PR #212; packed formats of stable-diffusion.cpp PR #2276):
- * ck_rotate_quant_rowwise_i8(bits=4) into `workspace`, then the GEMM of
- * ck_gemm_w4a4 reading those int8 codes against the packed int4 weights (same
- * results as ck_rotate_quant_rowwise + ck_gemm_w4a4).
- * K is the LOGICAL inner dimension (the packed weight has K/2 bytes per row).
+ * y = bf16(rotate-quantize(x) . W^T * scales (+ bias)), computed as
+ * ck_linear_w4a4_quantize followed by ck_linear_w4a4_matmul. Results equal
+ * ck_rotate_quant_rowwise(bits=4) followed by ck_gemm_w4a4 bit for bit.
+ * K is the LOGICAL inner dimension (the packed weight has K/2 bytes per row);
+ * K % 32 == 0 and K % group_size == 0.
  * workspace : device buffer of at least ck_linear_w4a4_workspace_bytes(M, K)
- *             bytes, 256-byte aligned; its contents are scratch.
- * Other arguments as above.
+ *             bytes, 256-byte aligned; opaque scratch written by the quantize
+ *             phase and read by the matmul phase.
+ * Other arguments as for ck_rotate_quant_rowwise and ck_gemm_w4a4.
  */
 ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N,
                          int64_t ldx, int group_size, const uint8_t* w_packed,
                          const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
                          void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The two phases of ck_linear_w4a4, callable separately (to time or overlap
+ * them). Phase 1 rotates and quantizes x into `workspace` (the int4 codes
+ * stored one per byte, as comfy-kitchen PR #212 "Related work" notes #201
+ * does away with the activation pack/unpack, in the column order the GEMM's
+ * weight decode produces, with the row scales and the row sums of the codes).
+ * Phase 2 runs the tensor-core GEMM of those codes against the packed int4
+ * weights and the rowwise-scale epilogue.
+ */
+ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                  int group_size, void* workspace, size_t ws_bytes, void* stream);
+ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed,
+                                const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                                const void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * W4A8 decode GEMV ("W4A8 decode GEMV" of comfy-kitchen PR #182, Description;

@@ -44,9 +44,9 @@ def test_version_and_last_error(ck):
 
 
 def test_workspace_bytes(ck):
-    # int8 activation codes (rounded up to 256 bytes), then float32 scales
-    assert ck.linear_w4a4_workspace_bytes(8192, 3840) == 8192 * 3840 + 8192 * 4
-    assert ck.linear_w4a4_workspace_bytes(3, 64) == 256 + 12
+    # int8 activation codes, float32 scales, int32 row sums (each rounded up to 256 bytes)
+    assert ck.linear_w4a4_workspace_bytes(8192, 3840) == 8192 * 3840 + 8192 * 4 + 8192 * 4
+    assert ck.linear_w4a4_workspace_bytes(3, 64) == 256 + 256 + 12
     assert ck.linear_w4a4_workspace_bytes(0, 64) == 0
 
 
@@ -87,6 +87,17 @@ def test_gemm_and_linear_validation(ck):
                             P(1 << 20), 16, None) == ck.CK_ERR_INVALID_ARG
     assert L.ck_linear_w4a4(P(1 << 20), 0, 8, 64, 8, 64, 64, P(1 << 20), P(1 << 20), None, P(1 << 20),
                             P((1 << 20) + 16), 1 << 20, None) == ck.CK_ERR_INVALID_ARG
+
+
+def test_linear_phase_validation(ck):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    ws = ck.linear_w4a4_workspace_bytes(8, 64)
+    assert L.ck_linear_w4a4_quantize(P(1 << 20), 0, 8, 64, 64, 64, P(1 << 21), ws - 1, None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_linear_w4a4_quantize(P(1 << 20), 0, 8, 64, 64, 48, P(1 << 21), ws, None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_linear_w4a4_quantize(P(1 << 20), 0, 8, 48, 48, 16, P(1 << 21), ws, None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_linear_w4a4_matmul(8, 64, 8, None, P(1 << 20), None, P(1 << 20), P(1 << 21), ws, None) == ck.CK_ERR_INVALID_ARG
+    assert L.ck_linear_w4a4_matmul(8, 64, 8, P(1 << 20), P(1 << 20), None, P(1 << 20), P((1 << 21) + 128), ws, None) == ck.CK_ERR_INVALID_ARG
 
 
 def test_predecoded_path_validation(ck):

@@ -243,6 +243,39 @@ def test_linear_w4a4_matches_oracle(ck, M, K, N, G, bias, dtype):
     assert_out_close(to_np_f64(y), O.bf16_bits_to_f64(r["y_bits"]))
 
 
+def _a256(v):
+    return (v + 255) // 256 * 256
+
+
+def _linear_workspace(ws, M, K):
+    """(codes in natural column order, scales, row sums) from the linear's workspace."""
+    nq = _a256(M * K)
+    q = ws[:M * K].view(torch.int8).view(M, K).cpu().numpy().astype(np.int64)
+    perm = np.array([0, 2, 4, 6, 1, 3, 5, 7])
+    nat = np.empty_like(q)
+    for j in range(8):
+        nat[:, perm[j]::8] = q[:, j::8]
+    s = ws[nq:nq + 4 * M].view(torch.float32).cpu().numpy()
+    rs = ws[nq + _a256(4 * M):nq + _a256(4 * M) + 4 * M].view(torch.int32).cpu().numpy()
+    return nat, s, rs
+
+
+def test_linear_phases_equal_rotate_quant_plus_gemm_w4a4(ck):
+    d = WL.small_linear_inputs(300, 1024, 520, seed=11, n_outlier_cols=10, with_bias=True)
+    x, wp, sw, b = d["x"].to(DEV), d["w_packed"].to(DEV), d["w_scale"].to(DEV), d["bias"].to(DEV)
+    ws = torch.empty(ck.linear_w4a4_workspace_bytes(300, 1024), device=DEV, dtype=torch.uint8)
+    ck.linear_w4a4_quantize(x, 64, ws)
+    y2 = ck.linear_w4a4_matmul(300, 1024, wp, sw, ws, bias=b)
+    y1 = ck.linear_w4a4(x, wp, sw, 64, bias=b)
+    qp, sp = ck.rotate_quant_rowwise(x, 64, 4)
+    y0 = ck.gemm_w4a4(qp, sp, wp, sw, bias=b)
+    assert torch.equal(y1, y0) and torch.equal(y2, y0)
+    q, s, rs = _linear_workspace(ws, 300, 1024)
+    np.testing.assert_array_equal(q, unpack_codes(qp))
+    np.testing.assert_array_equal(s, sp.cpu().numpy())
+    np.testing.assert_array_equal(rs, q.sum(axis=1))
+
+
 def _linear_full_config(ck, w, sample_rows):
     d = WL.linear_inputs(w)
     x, wp, sw = d["x"].to(DEV), d["w_packed"].to(DEV), d["w_scale"].to(DEV)
@@ -251,12 +284,12 @@ def _linear_full_config(ck, w, sample_rows):
     torch.cuda.synchronize()
     rows = np.asarray(sample_rows)
     r = O.linear_w4a4(to_np_f64(d["x"][rows]), d["w_packed"].numpy(), to_np_f64(d["w_scale"]), w.G)
-    # the quantized activations the GEMM consumed (workspace: int8 codes, then scales)
-    nq = w.M * w.K
-    qa = ws[:nq].view(torch.int8).view(w.M, w.K).cpu().numpy()[rows].astype(np.int64)
-    off = (nq + 255) // 256 * 256
-    sa = ws[off:off + 4 * w.M].view(torch.float32).cpu().numpy()[rows]
+    # the quantized activations the GEMM consumed (workspace: int8 codes with each 8-column group
+    # stored as columns (0 2 4 6 1 3 5 7), row scales, row sums of the codes)
+    qa, sa, rs = _linear_workspace(ws, w.M, w.K)
+    qa, sa, rs = qa[rows], sa[rows], rs[rows]
     assert qa.min() >= -7 and qa.max() <= 7
+    np.testing.assert_array_equal(rs, qa.sum(axis=1))
     assert_codes_close(qa, r["q"])
     assert_scales_close(sa, r["s"])
     rel = assert_out_close(to_np_f64(y.cpu()[rows]), O.bf16_bits_to_f64(r["y_bits"]))
