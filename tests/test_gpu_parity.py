@@ -122,7 +122,7 @@ def test_rotate_quant_mlp_down_G16_full(ck):
 
 
 @pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("G,K", [(64, 3840), (16, 1000), (256, 512)])
+@pytest.mark.parametrize("G,K", [(64, 3840), (16, 1008), (256, 512)])
 def test_rotate_quant_i8_codes_equal_packed_codes(ck, G, K, bits):
     M = 70
     xf = _rand_x(M, K, seed=K + bits, outliers=3)
