@@ -28,7 +28,7 @@ from . import workloads as WL
 
 
 def build_case(name: str, dev):
-    if name.startswith(("rq_", "gemm_", "linear_")):
+    if name.startswith(("rq_", "gemm_", "lin")):
         w = WL.LINEAR_M8192
         if name == "rq_M8192_K10240_G16":
             x = WL.linear_inputs(WL.LINEAR_MLP_DOWN)["x"].to(dev)
