@@ -105,8 +105,15 @@ template <int QBITS, int STORE, typename T>
 void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s, int32_t* rs, int nt,
                cudaStream_t st) {
   const float rnorm = (float)(1.0 / std::sqrt((double)G));
-  ck::rq::rotate_quant_kernel<QBITS, STORE, T><<<(unsigned)M, nt, 0, st>>>(
-      reinterpret_cast<const T*>(x), K, ldx, G, rnorm, reinterpret_cast<uint8_t*>(q), s, rs);
+  const T* xx = reinterpret_cast<const T*>(x);
+  uint8_t* qq = reinterpret_cast<uint8_t*>(q);
+  switch (G) {
+    case 1: ck::rq::rotate_quant_kernel<QBITS, STORE, 1, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
+    case 16: ck::rq::rotate_quant_kernel<QBITS, STORE, 16, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
+    case 64: ck::rq::rotate_quant_kernel<QBITS, STORE, 64, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
+    case 256: ck::rq::rotate_quant_kernel<QBITS, STORE, 256, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
+    default: ck::rq::rotate_quant_kernel<QBITS, STORE, 0, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
+  }
 }
 
 template <typename T>
@@ -198,6 +205,7 @@ ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const void*
   p.out = out;
   const size_t esz = EPI == EPI_I32 ? 4 : 2;
   p.out_vec_ok = aligned(out, 16) && ((N * (int64_t)esz) % 16 == 0);
+  p.col_vec_ok = (w_scale == nullptr || aligned(w_scale, 16)) && (bias == nullptr || aligned(bias, 16));
   const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
   const int pairs = (int)std::min<int64_t>(tiles, pairs_max);
 

@@ -74,8 +74,13 @@ struct Cfg {
   static constexpr bool BU = B_MODE == OP_PACKED4_U;
   static constexpr bool ANY_P = AP || BP;
   static constexpr bool ANY_I8 = !AP || !BP;
+  // With a decode path, the packed ring and the operand ring have the same
+  // depth and decode warp dw owns slot dw of both: every wait it makes is on
+  // the phase right after the one it saw last, so parity waits cannot alias.
   static constexpr int NU = !ANY_P ? 6 : ((AP && BP) ? 4 : 5);   // operand stages
-  static constexpr int NP = !ANY_P ? 1 : ((AP && BP) ? 5 : 6);   // packed stages
+  static constexpr int NP = !ANY_P ? 1 : NU;                      // packed stages
+  static constexpr int NDEC = ANY_P ? NU : 0;                     // active decode warps
+  static_assert(NDEC <= kDecWarps, "decode warps");
   static constexpr int P_STAGE = (AP ? A_P : 0) + (BP ? B_P : 0);
   static constexpr int I8_CTA_BYTES = (AP ? 0 : A_U) + (BP ? 0 : B_U);
   static constexpr int OFF_A = 0;
@@ -100,6 +105,7 @@ struct Params {
   const __nv_bfloat16* bias;      // (N) or null
   void* out;                      // (M, N) int32 or bf16
   int out_vec_ok;                 // 16-byte vector stores allowed
+  int col_vec_ok;                 // w_scale (and bias) 16-byte aligned: vector loads
 };
 
 // Writes one decoded 16-byte chunk (k = 16 * uc .. 16 * uc + 15 of the stage)
@@ -108,11 +114,11 @@ __device__ __forceinline__ void st_sw128(uint8_t* tile, int r, int uc, uint4 v) 
   *reinterpret_cast<uint4*>(tile + r * 128 + ((uc ^ (r & 7)) << 4)) = v;
 }
 
-// Decodes 128 packed rows (64 bytes each) of a stage into the operand tile.
+// One warp decodes 128 packed rows (64 bytes each) of a stage into the operand tile.
 template <bool UNSIGNED_PERM>
-__device__ __forceinline__ void decode_tile(const uint8_t* src, uint8_t* dst, int dt, int kbase, int K) {
-#pragma unroll
-  for (int c = dt; c < 128 * 4; c += kDecThreads) {
+__device__ __forceinline__ void decode_tile(const uint8_t* src, uint8_t* dst, int lane, int kbase, int K) {
+#pragma unroll 4
+  for (int c = lane; c < 128 * 4; c += 32) {
     const int r = c >> 2, pc = c & 3;
     uint4 o0 = make_uint4(0, 0, 0, 0), o1 = o0;
     if (kbase + pc * 32 < K) {   // columns past K decode to 0 (unsigned: weight 8 against code 0)
@@ -158,10 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NP; ++s) {
       mbar_init(&full_p[s], 1);
-      mbar_init(&empty_p[s], kDecWarps);
+      mbar_init(&empty_p[s], 1);
     }
     for (int s = 0; s < NU; ++s) {
-      mbar_init(&full_u[s], (C::ANY_P ? 2 * kDecWarps : 0) + (C::ANY_I8 ? 1 : 0));
+      mbar_init(&full_u[s], (C::ANY_P ? 2 : 0) + (C::ANY_I8 ? 1 : 0));
       mbar_init(&empty_u[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -261,23 +267,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < W_EPI0) {
     // ------------------------------------------------- decode (warps 2..9)
-    if (C::ANY_P) {
-      const int dt = threadIdx.x - W_DEC0 * 32;
+    // Stage g belongs to decode warp g % NU (slot g % NU of both rings): each
+    // warp turns a whole stage around (one proxy fence and one arrive per
+    // stage), and up to NU stages are decoded concurrently by different warps.
+    const int dw = warp - W_DEC0;
+    if (C::ANY_P && dw < C::NDEC) {
       int g = 0;
       bool ok = true;
       for (int t = pair; t < ntiles && ok; t += npairs) {
         for (int kb = 0; kb < nkb; ++kb, ++g) {
+          if (g % NU != dw) continue;
           const int sp = g % NP, su = g % NU;
           if (!warp_wait(&full_p[sp], (g / NP) & 1, abort, 6)) { ok = false; break; }
           if (!warp_wait(&empty_u[su], ((g / NU) & 1) ^ 1, abort, 7)) { ok = false; break; }
           const uint8_t* st = pk + sp * C::P_STAGE;
-          if (C::BP) decode_tile<C::BU>(st + (C::AP ? A_P : 0), b_u + su * B_U, dt, kb * BK, p.K);
-          if (C::AP) decode_tile<false>(st, a_u + su * A_U, dt, kb * BK, p.K);
+          if (C::BP) decode_tile<C::BU>(st + (C::AP ? A_P : 0), b_u + su * B_U, lane, kb * BK, p.K);
+          if (C::AP) decode_tile<false>(st, a_u + su * A_U, lane, kb * BK, p.K);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(&empty_p[sp]);
-            mbar_arrive_remote(mapa_shared(smem_u32(&full_u[su]), 0));
+            if (rank == 0) mbar_arrive(&full_u[su]);
+            else mbar_arrive_remote(mapa_shared(smem_u32(&full_u[su]), 0));
           }
         }
       }
@@ -318,18 +329,38 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (nb + j < p.N) orow[j] = (int32_t)r[j] - corr;
           }
         } else {
+          // per-column scale and bias of this chunk, as bf16 pairs (broadcast loads)
+          uint32_t cs[16], cb[16];
+          if (full && p.col_vec_ok) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.w_scale + nb) + j);
+              cs[4 * j] = a.x; cs[4 * j + 1] = a.y; cs[4 * j + 2] = a.z; cs[4 * j + 3] = a.w;
+              const uint4 b = has_bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + nb) + j) : make_uint4(0, 0, 0, 0);
+              cb[4 * j] = b.x; cb[4 * j + 1] = b.y; cb[4 * j + 2] = b.z; cb[4 * j + 3] = b.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = nb + 2 * j;
+              const uint32_t s0 = n < p.N ? __bfloat16_as_ushort(p.w_scale[n]) : 0u;
+              const uint32_t s1 = n + 1 < p.N ? __bfloat16_as_ushort(p.w_scale[n + 1]) : 0u;
+              const uint32_t b0 = (has_bias && n < p.N) ? __bfloat16_as_ushort(p.bias[n]) : 0u;
+              const uint32_t b1 = (has_bias && n + 1 < p.N) ? __bfloat16_as_ushort(p.bias[n + 1]) : 0u;
+              cs[j] = s0 | (s1 << 16);
+              cb[j] = b0 | (b1 << 16);
+            }
+          }
           uint32_t h[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const int n = nb + j;
-            const bool in0 = n < p.N, in1 = n + 1 < p.N;
-            const float sw0 = in0 ? __bfloat162float(p.w_scale[n]) : 0.0f;
-            const float sw1 = in1 ? __bfloat162float(p.w_scale[n + 1]) : 0.0f;
+            const float sw0 = __uint_as_float(cs[j >> 1] << 16);
+            const float sw1 = __uint_as_float(cs[j >> 1] & 0xFFFF0000u);
             float v0 = __fmul_rn(__fmul_rn((float)((int32_t)r[j] - corr), srow), sw0);
             float v1 = __fmul_rn(__fmul_rn((float)((int32_t)r[j + 1] - corr), srow), sw1);
             if (has_bias) {
-              v0 = __fadd_rn(v0, in0 ? __bfloat162float(p.bias[n]) : 0.0f);
-              v1 = __fadd_rn(v1, in1 ? __bfloat162float(p.bias[n + 1]) : 0.0f);
+              v0 = __fadd_rn(v0, __uint_as_float(cb[j >> 1] << 16));
+              v1 = __fadd_rn(v1, __uint_as_float(cb[j >> 1] & 0xFFFF0000u));
             }
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
             h[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);

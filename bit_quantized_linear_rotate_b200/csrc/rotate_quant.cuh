@@ -70,8 +70,15 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {       // a - b, one
   return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Sylvester butterflies on element-index bits below min(G, 32): for index bit h,
-// (a, b) -> (a + b, a - b) where a has the bit clear.
+// (a, b) -> (a + b, a - b) where a has the bit clear. G is a compile-time
+// constant for the common group sizes (the stage tests then vanish).
 __device__ __forceinline__ void fht_in_thread(float2 (&v)[EPT / 2], int G) {
   if (G > 1) {
 #pragma unroll
@@ -126,12 +133,15 @@ __device__ __forceinline__ float quant_exact(float y, float r, float s) {
   return e > 0.0f ? fl + 1.0f : (e < 0.0f ? fl : rintf(h));
 }
 
-template <int QBITS, int STORE, typename T>
+// GT: the group size when it is 1, 16, 64 or 256 (compile time), 0 otherwise
+// (then taken from G at run time).
+template <int QBITS, int STORE, int GT, typename T>
 __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict__ x, int K, int64_t ldx,
-                                                            int G, float rnorm, uint8_t* __restrict__ q,
+                                                            int G_rt, float rnorm, uint8_t* __restrict__ q,
                                                             float* __restrict__ scale,
                                                             int32_t* __restrict__ rowsum) {
   constexpr float kQmax = QBITS == 4 ? 7.0f : 127.0f;
+  const int G = GT ? GT : G_rt;
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
@@ -158,7 +168,7 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
   if (G > EPT) fht_across_lanes(v, G, lane);   // every lane runs it; columns past K hold zeros
   float amax = 0.0f;
 #pragma unroll
-  for (int e = 0; e < EPT / 2; ++e) amax = fmaxf(amax, fmaxf(fabsf(v[e].x), fabsf(v[e].y)));
+  for (int e = 0; e < EPT / 2; ++e) amax = max3(amax, fabsf(v[e].x), fabsf(v[e].y));
 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -188,11 +198,13 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
       u[2 * e + 1] = __float_as_uint(quant_exact(v[e].y, r, s) + magic);
     }
   } else {
-    const float rr = __fmul_rn(r, rnorm);          // exact for G = 4^k (rnorm a power of two)
+    // t = z * (r / sqrt(G)) + magic in one rounding: the nearest integer to the
+    // exact product (r / sqrt(G) is exact for G = 4^k)
+    const float rr = __fmul_rn(r, rnorm);
     const float2 r2 = make_float2(rr, rr), m2 = make_float2(magic, magic);
 #pragma unroll
     for (int e = 0; e < EPT / 2; ++e) {
-      const float2 t = __fadd2_rn(__fmul2_rn(v[e], r2), m2);
+      const float2 t = __ffma2_rn(v[e], r2, m2);
       u[2 * e] = __float_as_uint(t.x);
       u[2 * e + 1] = __float_as_uint(t.y);
     }
