@@ -101,6 +101,41 @@ ck_status ensure_smem_attr(KernelT kernel, size_t bytes) {
   return CK_OK;
 }
 
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+// Persistent grid: as many CTAs of `nt` threads as are co-resident (cached per kernel and nt).
+template <typename KernelT>
+unsigned persistent_grid(KernelT kern, int nt, int64_t work) {
+  static int cache_nt[64] = {0}, cache_blocks[64] = {0};
+  const int slot = (nt / 32) & 63;
+  int blocks = 0;
+  if (cache_nt[slot] == nt) {
+    blocks = cache_blocks[slot];
+  } else {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, nt, 0) != cudaSuccess || blocks <= 0) blocks = 1;
+    cache_blocks[slot] = blocks;
+    cache_nt[slot] = nt;
+  }
+  return (unsigned)std::min<int64_t>(work, (int64_t)blocks * sm_count());
+}
+
+template <int QBITS, int STORE, int GT, typename T>
+void launch_rq_g(const T* x, int64_t M, int K, int64_t ldx, int G, float rnorm, uint8_t* q, float* s, int32_t* rs,
+                 int nt, cudaStream_t st) {
+  auto kern = ck::rq::rotate_quant_kernel<QBITS, STORE, GT, T>;
+  kern<<<persistent_grid(kern, nt, M), nt, 0, st>>>(x, M, K, ldx, G, rnorm, q, s, rs);
+}
+
 template <int QBITS, int STORE, typename T>
 void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s, int32_t* rs, int nt,
                cudaStream_t st) {
@@ -108,11 +143,11 @@ void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, flo
   const T* xx = reinterpret_cast<const T*>(x);
   uint8_t* qq = reinterpret_cast<uint8_t*>(q);
   switch (G) {
-    case 1: ck::rq::rotate_quant_kernel<QBITS, STORE, 1, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
-    case 16: ck::rq::rotate_quant_kernel<QBITS, STORE, 16, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
-    case 64: ck::rq::rotate_quant_kernel<QBITS, STORE, 64, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
-    case 256: ck::rq::rotate_quant_kernel<QBITS, STORE, 256, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
-    default: ck::rq::rotate_quant_kernel<QBITS, STORE, 0, T><<<(unsigned)M, nt, 0, st>>>(xx, K, ldx, G, rnorm, qq, s, rs); break;
+    case 1: launch_rq_g<QBITS, STORE, 1, T>(xx, M, K, ldx, G, rnorm, qq, s, rs, nt, st); break;
+    case 16: launch_rq_g<QBITS, STORE, 16, T>(xx, M, K, ldx, G, rnorm, qq, s, rs, nt, st); break;
+    case 64: launch_rq_g<QBITS, STORE, 64, T>(xx, M, K, ldx, G, rnorm, qq, s, rs, nt, st); break;
+    case 256: launch_rq_g<QBITS, STORE, 256, T>(xx, M, K, ldx, G, rnorm, qq, s, rs, nt, st); break;
+    default: launch_rq_g<QBITS, STORE, 0, T>(xx, M, K, ldx, G, rnorm, qq, s, rs, nt, st); break;
   }
 }
 

@@ -33,7 +33,10 @@
 // 16-byte chunk c of row r at chunk c ^ (r % 8)).
 //
 // Warps: 0 packed-tile TMA producer, 1 MMA issue (even CTA) and TMEM
-// allocation, 2..9 nibble decode, 10..13 epilogue, 14 int8-tile TMA producer.
+// allocation, 2..11 nibble decode (two per operand slot, 64 rows each; the
+// first of each pair also issues that slot's int8-tile TMA as soon as the slot
+// is free; without a decode path warp 2 issues all int8 tiles), 12..15
+// epilogue.
 // TMEM holds two accumulators (2 x 256 columns): the epilogue of one tile
 // overlaps the main loop of the next. Every barrier wait is bounded
 // (ck_common.cuh); on a timeout the CTA stops issuing, drains what it issued,
@@ -57,10 +60,10 @@ constexpr int A_U = BM * BK;       // 16 KiB
 constexpr int B_U = BNH * BK;      // 16 KiB
 constexpr int A_P = BM * PKB;      // 8 KiB
 constexpr int B_P = BNH * PKB;     // 8 KiB
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 10;       // two per operand slot (at most 5 slots with a decode path)
 constexpr int kEpiWarps = 4;
-constexpr int W_PACK = 0, W_MMA = 1, W_DEC0 = 2, W_EPI0 = W_DEC0 + kDecWarps, W_I8 = W_EPI0 + kEpiWarps;
-constexpr int kThreads = (W_I8 + 1) * 32;
+constexpr int W_PACK = 0, W_MMA = 1, W_DEC0 = 2, W_EPI0 = W_DEC0 + kDecWarps;
+constexpr int kThreads = (W_EPI0 + kEpiWarps) * 32;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 
@@ -79,7 +82,7 @@ struct Cfg {
   // the phase right after the one it saw last, so parity waits cannot alias.
   static constexpr int NU = !ANY_P ? 6 : ((AP && BP) ? 4 : 5);   // operand stages
   static constexpr int NP = !ANY_P ? 1 : NU;                      // packed stages
-  static constexpr int NDEC = ANY_P ? NU : 0;                     // active decode warps
+  static constexpr int NDEC = ANY_P ? 2 * NU : 0;                 // active decode warps (2 per slot)
   static_assert(NDEC <= kDecWarps, "decode warps");
   static constexpr int P_STAGE = (AP ? A_P : 0) + (BP ? B_P : 0);
   static constexpr int I8_CTA_BYTES = (AP ? 0 : A_U) + (BP ? 0 : B_U);
@@ -114,17 +117,23 @@ __device__ __forceinline__ void st_sw128(uint8_t* tile, int r, int uc, uint4 v) 
   *reinterpret_cast<uint4*>(tile + r * 128 + ((uc ^ (r & 7)) << 4)) = v;
 }
 
-// One warp decodes 128 packed rows (64 bytes each) of a stage into the operand tile.
+// One warp decodes 64 packed rows (64 bytes each, rows [64 h, 64 h + 64)) of a
+// stage into the operand tile: all eight 16-byte loads are issued first.
 template <bool UNSIGNED_PERM>
-__device__ __forceinline__ void decode_tile(const uint8_t* src, uint8_t* dst, int lane, int kbase, int K) {
-#pragma unroll 4
-  for (int c = lane; c < 128 * 4; c += 32) {
-    const int r = c >> 2, pc = c & 3;
+__device__ __forceinline__ void decode_half(const uint8_t* src, uint8_t* dst, int h, int lane, int kbase, int K) {
+  uint4 pk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = 256 * h + 32 * i + lane, r = c >> 2, pc = c & 3;
+    pk[i] = *reinterpret_cast<const uint4*>(src + r * PKB + pc * 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = 256 * h + 32 * i + lane, r = c >> 2, pc = c & 3;
     uint4 o0 = make_uint4(0, 0, 0, 0), o1 = o0;
     if (kbase + pc * 32 < K) {   // columns past K decode to 0 (unsigned: weight 8 against code 0)
-      const uint4 pk = *reinterpret_cast<const uint4*>(src + r * PKB + pc * 16);
-      if (UNSIGNED_PERM) decode_nibbles_u8_perm(pk, o0, o1);
-      else decode_nibbles_s8(pk, o0, o1);
+      if (UNSIGNED_PERM) decode_nibbles_u8_perm(pk[i], o0, o1);
+      else decode_nibbles_s8(pk[i], o0, o1);
     }
     st_sw128(dst, r, 2 * pc, o0);
     st_sw128(dst, r, 2 * pc + 1, o1);
@@ -164,10 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NP; ++s) {
       mbar_init(&full_p[s], 1);
-      mbar_init(&empty_p[s], 1);
+      mbar_init(&empty_p[s], 2);
     }
     for (int s = 0; s < NU; ++s) {
-      mbar_init(&full_u[s], (C::ANY_P ? 2 : 0) + (C::ANY_I8 ? 1 : 0));
+      mbar_init(&full_u[s], (C::ANY_P ? 4 : 0) + (C::ANY_I8 ? 1 : 0));
       mbar_init(&empty_u[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -178,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if ((warp == W_PACK || warp == W_I8) && lane == 0) {
+  if ((warp == W_PACK || warp == W_DEC0) && lane == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
   }
@@ -214,27 +223,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = g - 1; h >= 0 && h >= g - NP; --h)
           mbar_wait(&full_p[h % NP], (h / NP) & 1, nullptr, 3, 100000000ull);
     }
-  } else if (warp == W_I8) {
-    // --------------------------------------------------- int8-tile producer
-    if (C::ANY_I8 && lane == 0) {
-      int g = 0;
-      bool ok = true;
-      for (int t = pair; t < ntiles && ok; t += npairs) {
-        const int m_row = (t / p.tiles_n) * 256 + (int)rank * BM;
-        const int n_row = (t % p.tiles_n) * BN + (int)rank * BNH;
-        for (int kb = 0; kb < nkb; ++kb, ++g) {
-          const int su = g % NU;
-          if (!mbar_wait(&empty_u[su], ((g / NU) & 1) ^ 1, abort, 2)) { ok = false; break; }
-          if (rank == 0) mbar_arrive_expect_tx(&full_u[su], 2 * C::I8_CTA_BYTES);
-          const uint32_t bar = mapa_shared(smem_u32(&full_u[su]), 0);
-          if (!C::AP) tma_load_2d_pair(a_u + su * A_U, &tm_a, bar, kb * BK, m_row);
-          if (!C::BP) tma_load_2d_pair(b_u + su * B_U, &tm_b, bar, kb * BK, n_row);
-        }
-      }
-      if (!ok && rank == 0)   // drain (the leader's barrier counts both CTAs' bytes)
-        for (int h = g - 1; h >= 0 && h >= g - NU; --h)
-          mbar_wait_cluster(&full_u[h % NU], (h / NU) & 1, nullptr, 3, 100000000ull);
-    }
   } else if (warp == W_MMA) {
     // ------------------------------------------------ MMA issue (leader CTA)
     if (rank == 0 && lane == 0) {
@@ -266,23 +254,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp < W_EPI0) {
-    // ------------------------------------------------- decode (warps 2..9)
-    // Stage g belongs to decode warp g % NU (slot g % NU of both rings): each
-    // warp turns a whole stage around (one proxy fence and one arrive per
-    // stage), and up to NU stages are decoded concurrently by different warps.
+    // ------------------------------------------------ decode (warps 2..11)
+    // Stage g belongs to the decode warps 2 (g % NU) and 2 (g % NU) + 1 (slot
+    // g % NU of both rings), each taking half of the rows: a pair of warps
+    // turns a whole stage around (one proxy fence and one arrive per warp and
+    // stage), and up to NU stages are decoded concurrently.
     const int dw = warp - W_DEC0;
     if (C::ANY_P && dw < C::NDEC) {
-      int g = 0;
+      const int half = dw & 1, slot = dw >> 1;
+      int g = 0, last_i8 = -1;
       bool ok = true;
       for (int t = pair; t < ntiles && ok; t += npairs) {
+        const int m_row = (t / p.tiles_n) * 256 + (int)rank * BM;
+        const int n_row = (t % p.tiles_n) * BN + (int)rank * BNH;
         for (int kb = 0; kb < nkb; ++kb, ++g) {
-          if (g % NU != dw) continue;
+          if (g % NU != slot) continue;
           const int sp = g % NP, su = g % NU;
-          if (!warp_wait(&full_p[sp], (g / NP) & 1, abort, 6)) { ok = false; break; }
           if (!warp_wait(&empty_u[su], ((g / NU) & 1) ^ 1, abort, 7)) { ok = false; break; }
+          if (C::ANY_I8 && half == 0 && lane == 0) {   // the slot is free: fetch its int8 tiles
+            if (rank == 0) mbar_arrive_expect_tx(&full_u[su], 2 * C::I8_CTA_BYTES);
+            const uint32_t bar = mapa_shared(smem_u32(&full_u[su]), 0);
+            if (!C::AP) tma_load_2d_pair(a_u + su * A_U, &tm_a, bar, kb * BK, m_row);
+            if (!C::BP) tma_load_2d_pair(b_u + su * B_U, &tm_b, bar, kb * BK, n_row);
+            last_i8 = g;
+          }
+          if (!warp_wait(&full_p[sp], (g / NP) & 1, abort, 6)) { ok = false; break; }
           const uint8_t* st = pk + sp * C::P_STAGE;
-          if (C::BP) decode_tile<C::BU>(st + (C::AP ? A_P : 0), b_u + su * B_U, lane, kb * BK, p.K);
-          if (C::AP) decode_tile<false>(st, a_u + su * A_U, lane, kb * BK, p.K);
+          if (C::BP) decode_half<C::BU>(st + (C::AP ? A_P : 0), b_u + su * B_U, half, lane, kb * BK, p.K);
+          if (C::AP) decode_half<false>(st, a_u + su * A_U, half, lane, kb * BK, p.K);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -292,9 +291,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (!ok && rank == 0 && lane == 0 && last_i8 >= 0)   // drain the int8 tiles this warp requested
+        mbar_wait_cluster(&full_u[last_i8 % NU], (last_i8 / NU) & 1, nullptr, 3, 100000000ull);
+    } else if (!C::ANY_P && dw == 0 && lane == 0) {
+      // ------------------------------------------- int8-tile producer (no decode path)
+      int g = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        const int m_row = (t / p.tiles_n) * 256 + (int)rank * BM;
+        const int n_row = (t % p.tiles_n) * BN + (int)rank * BNH;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int su = g % NU;
+          if (!mbar_wait(&empty_u[su], ((g / NU) & 1) ^ 1, abort, 2)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&full_u[su], 2 * C::I8_CTA_BYTES);
+          const uint32_t bar = mapa_shared(smem_u32(&full_u[su]), 0);
+          tma_load_2d_pair(a_u + su * A_U, &tm_a, bar, kb * BK, m_row);
+          tma_load_2d_pair(b_u + su * B_U, &tm_b, bar, kb * BK, n_row);
+        }
+      }
+      if (!ok && rank == 0)   // drain (the leader's barrier counts both CTAs' bytes)
+        for (int h = g - 1; h >= 0 && h >= g - NU; --h)
+          mbar_wait_cluster(&full_u[h % NU], (h / NU) & 1, nullptr, 3, 100000000ull);
     }
-  } else if (warp < W_I8) {
-    // ------------------------------------------------ epilogue (warps 10..13)
+  } else {
+    // ------------------------------------------------ epilogue (warps 12..15)
     const int quarter = warp & 3;               // TMEM lanes this warp may read
     const int rl = quarter * 32 + lane;         // accumulator row of this thread
     const bool has_bias = p.bias != nullptr;
@@ -309,31 +329,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float srow = (EPI == EPI_BF16 && row_ok) ? p.a_scale[m] : 0.0f;
       const int corr = (C::BU && row_ok) ? 8 * p.a_rowsum[m] : 0;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + (uint32_t)(ab * BN) + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, r);
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem + (uint32_t)(ab * BN) + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, r);
         tmem_ld_wait();
         const int nb = n0 + c0;
         if (!row_ok || nb >= p.N) continue;
-        const bool full = (nb + 32 <= p.N) && p.out_vec_ok;
+        const bool full = (nb + 16 <= p.N) && p.out_vec_ok;
         if (EPI == EPI_I32) {
           int32_t* orow = reinterpret_cast<int32_t*>(p.out) + (int64_t)m * p.N + nb;
           if (full) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
+            for (int j = 0; j < 16; j += 4)
               *reinterpret_cast<uint4*>(orow + j) =
                   make_uint4(r[j] - corr, r[j + 1] - corr, r[j + 2] - corr, r[j + 3] - corr);
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
+            for (int j = 0; j < 16; ++j)
               if (nb + j < p.N) orow[j] = (int32_t)r[j] - corr;
           }
         } else {
-          // per-column scale and bias of this chunk, as bf16 pairs (broadcast loads)
-          uint32_t cs[16], cb[16];
+          // per-column scale and bias of these 16 columns, as bf16 pairs (broadcast loads)
+          uint32_t cs[8], cb[8];
           if (full && p.col_vec_ok) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
               const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.w_scale + nb) + j);
               cs[4 * j] = a.x; cs[4 * j + 1] = a.y; cs[4 * j + 2] = a.z; cs[4 * j + 3] = a.w;
               const uint4 b = has_bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + nb) + j) : make_uint4(0, 0, 0, 0);
@@ -341,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 8; ++j) {
               const int n = nb + 2 * j;
               const uint32_t s0 = n < p.N ? __bfloat16_as_ushort(p.w_scale[n]) : 0u;
               const uint32_t s1 = n + 1 < p.N ? __bfloat16_as_ushort(p.w_scale[n + 1]) : 0u;
@@ -351,9 +371,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               cb[j] = b0 | (b1 << 16);
             }
           }
-          uint32_t h[16];
+          uint32_t hh[8];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
+          for (int j = 0; j < 16; j += 2) {
             const float sw0 = __uint_as_float(cs[j >> 1] << 16);
             const float sw1 = __uint_as_float(cs[j >> 1] & 0xFFFF0000u);
             float v0 = __fmul_rn(__fmul_rn((float)((int32_t)r[j] - corr), srow), sw0);
@@ -363,18 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               v1 = __fadd_rn(v1, __uint_as_float(cb[j >> 1] & 0xFFFF0000u));
             }
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-            h[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+            hh[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
           }
           __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)m * p.N + nb;
           if (full) {
-#pragma unroll
-            for (int j = 0; j < 16; j += 4)
-              *reinterpret_cast<uint4*>(orow + 2 * j) = make_uint4(h[j], h[j + 1], h[j + 2], h[j + 3]);
+            *reinterpret_cast<uint4*>(orow) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+            *reinterpret_cast<uint4*>(orow + 8) = make_uint4(hh[4], hh[5], hh[6], hh[7]);
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
               if (nb + j < p.N) {
-                const uint32_t hw = h[j >> 1];
+                const uint32_t hw = hh[j >> 1];
                 reinterpret_cast<unsigned short*>(orow)[j] =
                     (j & 1) ? (unsigned short)(hw >> 16) : (unsigned short)(hw & 0xFFFFu);
               }

@@ -6,8 +6,9 @@
 // warp-shuffle Hadamard transform as in the CUDA INT8 rowwise ConvRot quantizer
 // named by comfy-kitchen PR #182 ("Description").
 //
-// One CTA per row; thread t owns the 32 contiguous columns [32t, 32t + 32)
-// (four 128-bit loads). The transform runs in fp32: log2(min(G, 32)) butterfly
+// A persistent grid of CTAs walks the rows, one row per CTA at a time, the next
+// row's loads issued before the current row is processed; thread t owns the 32
+// contiguous columns [32t, 32t + 32) (four 128-bit loads). The transform runs in fp32: log2(min(G, 32)) butterfly
 // stages inside the thread, then log2(G / 32) stages across lanes
 // (__shfl_xor_sync, one shuffle and one FMA per element and stage), then the
 // 1/sqrt(G) normalisation (a power of two for G = 16, 64, 256). The rotated row
@@ -38,12 +39,18 @@ constexpr int EPT = 32;   // columns per thread
 // nibbles without byte shuffles).
 enum Store { STORE_PACKED4 = 0, STORE_INT8 = 1, STORE_INT8_PERM = 2 };
 
+// Raw 128-bit loads of a thread's 32 columns (4 x 8 values), zero past K.
+__device__ __forceinline__ void load_raw(const void* row, int e0, int K, uint4 (&raw)[EPT / 8]) {
+#pragma unroll
+  for (int j = 0; j < EPT / 8; ++j)
+    raw[j] = (e0 + 8 * j < K) ? __ldcs(reinterpret_cast<const uint4*>(row) + (e0 / 8 + j)) : make_uint4(0, 0, 0, 0);
+}
+
 template <typename T>
-__device__ __forceinline__ void load8(const T* p, float* f);
+__device__ __forceinline__ void to_float8(const uint4 raw, float* f);
 
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
-  const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void to_float8<__nv_bfloat16>(const uint4 raw, float* f) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -53,8 +60,7 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
 }
 
 template <>
-__device__ __forceinline__ void load8<__half>(const __half* p, float* f) {
-  const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void to_float8<__half>(const uint4 raw, float* f) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -136,131 +142,130 @@ __device__ __forceinline__ float quant_exact(float y, float r, float s) {
 // GT: the group size when it is 1, 16, 64 or 256 (compile time), 0 otherwise
 // (then taken from G at run time).
 template <int QBITS, int STORE, int GT, typename T>
-__global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict__ x, int K, int64_t ldx,
+__global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
                                                             int G_rt, float rnorm, uint8_t* __restrict__ q,
                                                             float* __restrict__ scale,
                                                             int32_t* __restrict__ rowsum) {
   constexpr float kQmax = QBITS == 4 ? 7.0f : 127.0f;
   const int G = GT ? GT : G_rt;
-  __shared__ float red[32];
-  const int64_t row = blockIdx.x;
+  __shared__ float red[4][32];   // [2 * (it & 1)]: amax, [2 * (it & 1) + 1]: row sum
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int e0 = tid * EPT;
-  const T* xr = x + row * ldx;
 
-  float2 v[EPT / 2];
+  // persistent over rows; the next row's 128-bit loads are in flight while
+  // the current row is transformed, reduced and quantized
+  int64_t row = blockIdx.x;
+  uint4 raw[EPT / 8];
+  if (row < M) load_raw(x + row * ldx, e0, K, raw);
+  for (int it = 0; row < M; row += gridDim.x, ++it) {
+    float2 v[EPT / 2];
 #pragma unroll
-  for (int j = 0; j < EPT / 8; ++j) {
-    float f[8];
-    if (e0 + 8 * j < K) {
-      load8<T>(xr + e0 + 8 * j, f);
-    } else {
+    for (int j = 0; j < EPT / 8; ++j) {
+      float f[8];
+      to_float8<T>(raw[j], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+      for (int e = 0; e < 4; ++e) v[4 * j + e] = make_float2(f[2 * e], f[2 * e + 1]);
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) v[4 * j + e] = make_float2(f[2 * e], f[2 * e + 1]);
-  }
+    const int64_t next = row + gridDim.x;
+    if (next < M) load_raw(x + next * ldx, e0, K, raw);
 
-  // unnormalised transform z = x H; the 1/sqrt(G) factor is folded into the scale
-  fht_in_thread(v, G);
-  if (G > EPT) fht_across_lanes(v, G, lane);   // every lane runs it; columns past K hold zeros
-  float amax = 0.0f;
+    // unnormalised transform z = x H; the 1/sqrt(G) factor is folded into the scale
+    fht_in_thread(v, G);
+    if (G > EPT) fht_across_lanes(v, G, lane);   // every lane runs it; columns past K hold zeros
+    float amax = 0.0f;
 #pragma unroll
-  for (int e = 0; e < EPT / 2; ++e) amax = max3(amax, fabsf(v[e].x), fabsf(v[e].y));
+    for (int e = 0; e < EPT / 2; ++e) amax = max3(amax, fabsf(v[e].x), fabsf(v[e].y));
 
+    // block reductions alternate between buffer pairs, so one barrier per reduction suffices
+    float* rb = red[2 * (it & 1)];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (lane == 0) red[tid >> 5] = amax;
-  __syncthreads();
-  if (tid < 32) {
-    float a = tid < (int)(blockDim.x >> 5) ? red[tid] : 0.0f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if (tid == 0) red[0] = a;
-  }
-  __syncthreads();
-  amax = __fmul_rn(red[0], rnorm);               // amax of y = z / sqrt(G)
-
-  // positive-scale contract: an all-zero row gets scale 1 and all-zero codes
-  const float s = amax > 0.0f ? __fdiv_rn(amax, kQmax) : 1.0f;
-  const float r = __frcp_rn(s);
-  if (tid == 0) scale[row] = s;
-
-  // codes: bit patterns whose low byte is q (int8) or q + 8 (offset-binary int4)
-  uint32_t u[EPT];
-  const float magic = STORE == STORE_PACKED4 ? kRoundMagic + 8.0f : kRoundMagic;
-  if (G == 1) {
-#pragma unroll
-    for (int e = 0; e < EPT / 2; ++e) {
-      u[2 * e] = __float_as_uint(quant_exact(v[e].x, r, s) + magic);
-      u[2 * e + 1] = __float_as_uint(quant_exact(v[e].y, r, s) + magic);
-    }
-  } else {
-    // t = z * (r / sqrt(G)) + magic in one rounding: the nearest integer to the
-    // exact product (r / sqrt(G) is exact for G = 4^k)
-    const float rr = __fmul_rn(r, rnorm);
-    const float2 r2 = make_float2(rr, rr), m2 = make_float2(magic, magic);
-#pragma unroll
-    for (int e = 0; e < EPT / 2; ++e) {
-      const float2 t = __ffma2_rn(v[e], r2, m2);
-      u[2 * e] = __float_as_uint(t.x);
-      u[2 * e + 1] = __float_as_uint(t.y);
-    }
-  }
-  // low bytes of four codes -> one word (natural order, or (0 2 4 6)(1 3 5 7) per 8 columns)
-  uint32_t g[EPT / 4];
-#pragma unroll
-  for (int j = 0; j < EPT / 4; ++j) {
-    const int b = STORE == STORE_INT8_PERM ? 8 * (j >> 1) + (j & 1) : 4 * j;
-    const int st = STORE == STORE_INT8_PERM ? 2 : 1;
-    g[j] = __byte_perm(__byte_perm(u[b], u[b + st], 0x5140), __byte_perm(u[b + 2 * st], u[b + 3 * st], 0x5140),
-                       0x5410);
-  }
-  if (STORE == STORE_INT8_PERM) {
-    int sum = 0;
-#pragma unroll
-    for (int j = 0; j < EPT / 4; ++j) sum = __dp4a((int)g[j], 0x01010101, sum);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    __syncthreads();                                  // red[] is free again
-    if (lane == 0) red[tid >> 5] = __int_as_float(sum);
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) rb[tid >> 5] = amax;
     __syncthreads();
-    if (tid < 32) {
-      int a = tid < (int)(blockDim.x >> 5) ? __float_as_int(red[tid]) : 0;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (tid == 0) rowsum[row] = a;
-    }
-  }
-  if (e0 >= K) return;
+    amax = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, rb[w]);
+    amax = __fmul_rn(amax, rnorm);               // amax of y = z / sqrt(G)
 
-  if (STORE == STORE_PACKED4) {
-    // bytes hold u = q + 8 < 16: fold neighbours into nibbles, low nibble = even column
-    uint32_t w[4];
+    // positive-scale contract: an all-zero row gets scale 1 and all-zero codes
+    const float s = amax > 0.0f ? __fdiv_rn(amax, kQmax) : 1.0f;
+    const float r = __frcp_rn(s);
+    if (tid == 0) scale[row] = s;
+
+    // codes: bit patterns whose low byte is q (int8) or q + 8 (offset-binary int4)
+    uint32_t u[EPT];
+    const float magic = STORE == STORE_PACKED4 ? kRoundMagic + 8.0f : kRoundMagic;
+    if (G == 1) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t ta = g[2 * j] | (g[2 * j] >> 4), tb = g[2 * j + 1] | (g[2 * j + 1] >> 4);
-      w[j] = __byte_perm(ta, tb, 0x6420);
-    }
-    uint8_t* qr = q + row * (int64_t)(K >> 1) + (e0 >> 1);
-    if ((K & 31) == 0) {          // rows of K/2 bytes are 16-byte aligned
-      *reinterpret_cast<uint4*>(qr) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int e = 0; e < EPT / 2; ++e) {
+        u[2 * e] = __float_as_uint(quant_exact(v[e].x, r, s) + magic);
+        u[2 * e + 1] = __float_as_uint(quant_exact(v[e].y, r, s) + magic);
+      }
     } else {
+      // t = z * (r / sqrt(G)) + magic in one rounding: the nearest integer to the
+      // exact product (r / sqrt(G) is exact for G = 4^k)
+      const float rr = __fmul_rn(r, rnorm);
+      const float2 r2 = make_float2(rr, rr), m2 = make_float2(magic, magic);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (e0 + 8 * j < K) reinterpret_cast<uint32_t*>(qr)[j] = w[j];
+      for (int e = 0; e < EPT / 2; ++e) {
+        const float2 t = __ffma2_rn(v[e], r2, m2);
+        u[2 * e] = __float_as_uint(t.x);
+        u[2 * e + 1] = __float_as_uint(t.y);
+      }
     }
-  } else {
-    uint8_t* qr = q + row * (int64_t)K + e0;
-    if ((K & 31) == 0) {
-      reinterpret_cast<uint4*>(qr)[0] = make_uint4(g[0], g[1], g[2], g[3]);
-      reinterpret_cast<uint4*>(qr)[1] = make_uint4(g[4], g[5], g[6], g[7]);
-    } else {
+    // low bytes of four codes -> one word (natural order, or (0 2 4 6)(1 3 5 7) per 8 columns)
+    uint32_t g[EPT / 4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (e0 + 8 * j < K) reinterpret_cast<uint2*>(qr)[j] = make_uint2(g[2 * j], g[2 * j + 1]);
+    for (int j = 0; j < EPT / 4; ++j) {
+      const int b = STORE == STORE_INT8_PERM ? 8 * (j >> 1) + (j & 1) : 4 * j;
+      const int st = STORE == STORE_INT8_PERM ? 2 : 1;
+      g[j] = __byte_perm(__byte_perm(u[b], u[b + st], 0x5140), __byte_perm(u[b + 2 * st], u[b + 3 * st], 0x5140),
+                         0x5410);
+    }
+    if (STORE == STORE_INT8_PERM) {
+      int sum = 0;
+#pragma unroll
+      for (int j = 0; j < EPT / 4; ++j) sum = __dp4a((int)g[j], 0x01010101, sum);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      float* rs = red[2 * (it & 1) + 1];
+      if (lane == 0) rs[tid >> 5] = __int_as_float(sum);
+      __syncthreads();
+      if (tid == 0) {
+        int a = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) a += __float_as_int(rs[w]);
+        rowsum[row] = a;
+      }
+    }
+
+    if (e0 < K) {
+      if (STORE == STORE_PACKED4) {
+        // bytes hold u = q + 8 < 16: fold neighbours into nibbles, low nibble = even column
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t ta = g[2 * j] | (g[2 * j] >> 4), tb = g[2 * j + 1] | (g[2 * j + 1] >> 4);
+          w[j] = __byte_perm(ta, tb, 0x6420);
+        }
+        uint8_t* qr = q + row * (int64_t)(K >> 1) + (e0 >> 1);
+        if ((K & 31) == 0) {          // rows of K/2 bytes are 16-byte aligned
+          *reinterpret_cast<uint4*>(qr) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (e0 + 8 * j < K) reinterpret_cast<uint32_t*>(qr)[j] = w[j];
+        }
+      } else {
+        uint8_t* qr = q + row * (int64_t)K + e0;
+        if ((K & 31) == 0) {
+          reinterpret_cast<uint4*>(qr)[0] = make_uint4(g[0], g[1], g[2], g[3]);
+          reinterpret_cast<uint4*>(qr)[1] = make_uint4(g[4], g[5], g[6], g[7]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (e0 + 8 * j < K) reinterpret_cast<uint2*>(qr)[j] = make_uint2(g[2 * j], g[2 * j + 1]);
+        }
+      }
     }
   }
 }
