@@ -113,16 +113,18 @@ int sm_count() {
   return cache[dev];
 }
 
-// Persistent grid: as many CTAs of `nt` threads as are co-resident (cached per kernel and nt).
-template <typename KernelT>
-unsigned persistent_grid(KernelT kern, int nt, int64_t work) {
+// Persistent grid: as many CTAs of `nt` threads (and `smem` dynamic bytes) as
+// are co-resident (cached per kernel instantiation, through Tag, and nt).
+template <typename Tag, typename KernelT>
+unsigned persistent_grid(KernelT kern, int nt, size_t smem, int64_t work) {
   static int cache_nt[64] = {0}, cache_blocks[64] = {0};
   const int slot = (nt / 32) & 63;
   int blocks = 0;
   if (cache_nt[slot] == nt) {
     blocks = cache_blocks[slot];
   } else {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, nt, 0) != cudaSuccess || blocks <= 0) blocks = 1;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, nt, smem) != cudaSuccess || blocks <= 0) blocks = 1;
     cache_blocks[slot] = blocks;
     cache_nt[slot] = nt;
   }
@@ -133,7 +135,9 @@ template <int QBITS, int STORE, int GT, typename T>
 void launch_rq_g(const T* x, int64_t M, int K, int64_t ldx, int G, float rnorm, uint8_t* q, float* s, int32_t* rs,
                  int nt, cudaStream_t st) {
   auto kern = ck::rq::rotate_quant_kernel<QBITS, STORE, GT, T>;
-  kern<<<persistent_grid(kern, nt, M), nt, 0, st>>>(x, M, K, ldx, G, rnorm, q, s, rs);
+  const size_t smem = (size_t)(nt / 32) * 2048;     // one 2 KB transpose buffer per warp
+  struct Tag {};
+  kern<<<persistent_grid<Tag>(kern, nt, smem, M), nt, smem, st>>>(x, M, K, ldx, G, rnorm, q, s, rs);
 }
 
 template <int QBITS, int STORE, typename T>

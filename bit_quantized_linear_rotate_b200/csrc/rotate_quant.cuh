@@ -39,11 +39,30 @@ constexpr int EPT = 32;   // columns per thread
 // nibbles without byte shuffles).
 enum Store { STORE_PACKED4 = 0, STORE_INT8 = 1, STORE_INT8_PERM = 2 };
 
-// Raw 128-bit loads of a thread's 32 columns (4 x 8 values), zero past K.
-__device__ __forceinline__ void load_raw(const void* row, int e0, int K, uint4 (&raw)[EPT / 8]) {
+// Coalesced 128-bit loads of the warp's 1024 columns: lane l takes 16-byte
+// chunks l, 32 + l, 64 + l, 96 + l of the warp's span (zero past K).
+__device__ __forceinline__ void load_raw(const void* row, int warp, int lane, int K, uint4 (&raw)[EPT / 8]) {
 #pragma unroll
-  for (int j = 0; j < EPT / 8; ++j)
-    raw[j] = (e0 + 8 * j < K) ? __ldcs(reinterpret_cast<const uint4*>(row) + (e0 / 8 + j)) : make_uint4(0, 0, 0, 0);
+  for (int j = 0; j < EPT / 8; ++j) {
+    const int c = 128 * warp + 32 * j + lane;           // 16-byte chunk index in the row
+    raw[j] = (8 * c < K) ? __ldcs(reinterpret_cast<const uint4*>(row) + c) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// 16-byte slot of chunk c in a warp's 2 KB transpose buffer: the low three bits
+// (position in a 128-byte line) are XORed with the line index, so both the
+// coalesced writes and the contiguous per-thread reads are bank-conflict free.
+__device__ __forceinline__ int tslot(int c) { return c ^ ((c >> 3) & 7); }
+
+// Regroups the coalesced chunks so that lane l holds chunks 4l .. 4l + 3 (its
+// 32 contiguous columns).
+__device__ __forceinline__ void transpose_raw(uint4* buf, int lane, uint4 (&raw)[EPT / 8]) {
+#pragma unroll
+  for (int j = 0; j < EPT / 8; ++j) buf[tslot(32 * j + lane)] = raw[j];
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < EPT / 8; ++j) raw[j] = buf[tslot(4 * lane + j)];
+  __syncwarp();
 }
 
 template <typename T>
@@ -149,16 +168,20 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
   constexpr float kQmax = QBITS == 4 ? 7.0f : 127.0f;
   const int G = GT ? GT : G_rt;
   __shared__ float red[4][32];   // [2 * (it & 1)]: amax, [2 * (it & 1) + 1]: row sum
+  extern __shared__ uint4 tbuf_all[];              // 2 KB per warp
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  const int warp = tid >> 5;
   const int e0 = tid * EPT;
+  uint4* tbuf = tbuf_all + 128 * warp;
 
   // persistent over rows; the next row's 128-bit loads are in flight while
   // the current row is transformed, reduced and quantized
   int64_t row = blockIdx.x;
   uint4 raw[EPT / 8];
-  if (row < M) load_raw(x + row * ldx, e0, K, raw);
+  if (row < M) load_raw(x + row * ldx, warp, lane, K, raw);
   for (int it = 0; row < M; row += gridDim.x, ++it) {
+    transpose_raw(tbuf, lane, raw);
     float2 v[EPT / 2];
 #pragma unroll
     for (int j = 0; j < EPT / 8; ++j) {
@@ -168,7 +191,7 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
       for (int e = 0; e < 4; ++e) v[4 * j + e] = make_float2(f[2 * e], f[2 * e + 1]);
     }
     const int64_t next = row + gridDim.x;
-    if (next < M) load_raw(x + next * ldx, e0, K, raw);
+    if (next < M) load_raw(x + next * ldx, warp, lane, K, raw);
 
     // unnormalised transform z = x H; the 1/sqrt(G) factor is folded into the scale
     fht_in_thread(v, G);
