@@ -17,6 +17,7 @@
 #include "ck_common.cuh"
 #include "gemm_w4a4_sm100.cuh"
 #include "gemv_awq.cuh"
+#include "gemv_stream.cuh"
 #include "gemv_w4a8.cuh"
 #include "rotate_quant.cuh"
 
@@ -69,21 +70,39 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major byte matrix (rows x cols) with row stride `ld` bytes, box = (box_cols x box_rows).
+// Row-major matrix (rows x cols elements of `dt`) with row stride `ld` bytes,
+// box = (box_cols x box_rows) elements.
 ck_status make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
-                    uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+                    uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw,
+                    CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(CK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {ld};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return CK_OK;
 }
+
+// Shared-memory layout of a streaming GEMV: as many stages as fit in ~200 KB.
+ck::gstream::Layout stream_layout(int stage_bytes, int misc_bytes) {
+  using namespace ck::gstream;
+  Layout L;
+  L.stage_bytes = (stage_bytes + 127) / 128 * 128;
+  const int red_stage = kCons * 32 * 4 * 4;
+  const int budget = 200 * 1024 - misc_bytes - 3 * kMaxStages * 8 - 256;
+  L.ns = std::min(kMaxStages, budget / (L.stage_bytes + red_stage));
+  L.off_red = L.ns * L.stage_bytes;
+  L.off_misc = L.off_red + L.ns * red_stage;
+  L.off_bar = (L.off_misc + misc_bytes + 15) / 16 * 16;
+  L.total = L.off_bar + 3 * kMaxStages * 8;
+  return L;
+}
+
 
 // ------------------------------------------------------------------ kernels
 
@@ -491,10 +510,36 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
   if (!aligned(xq, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: operands must be 16-byte aligned");
   if (!aligned(x_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "gemv_w4a8: misaligned scale, bias or output");
-  const unsigned grid = (unsigned)((N + ck::w4a8::kRows - 1) / ck::w4a8::kRows);
   const auto* sw = reinterpret_cast<const __nv_bfloat16*>(w_scale);
   const auto* bb = reinterpret_cast<const __nv_bfloat16*>(bias);
   auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
+  if (K <= 4096) {
+    // streaming path: 8-row weight tiles through a shared-memory ring, one CTA per SM
+    using namespace ck::gstream;
+    W4A8Params sp;
+    sp.xq = xq; sp.xs = x_scale; sp.w = w_packed; sp.sw = sw; sp.bias = bb; sp.y = yy;
+    sp.M = (int)M; sp.K = (int)K; sp.N = (int)N;
+    sp.ntiles = (int)((N + 7) / 8);
+    const int grid = std::min(sp.ntiles, sm_count());
+    const int tpc = (sp.ntiles + grid - 1) / grid;
+    sp.L = stream_layout(8 * (int)(K / 2), kCons * 16 * 4 + 2 * 8 * tpc * 4 + 16);
+    const int nchunk = (int)(K / 128), cpw = (nchunk + kCons - 1) / kCons;
+    cudaError_t e;
+#define CK_W4A8_STREAM(CPW)                                                                      \
+    {                                                                                            \
+      auto kern = w4a8_stream_kernel<CPW>;                                                       \
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sp.L.total);   \
+      if (e == cudaSuccess) kern<<<grid, kThreads, sp.L.total, S(stream)>>>(sp);                 \
+    }
+    if (cpw <= 1) CK_W4A8_STREAM(1)
+    else if (cpw == 2) CK_W4A8_STREAM(2)
+    else if (cpw == 3) CK_W4A8_STREAM(3)
+    else CK_W4A8_STREAM(4)
+#undef CK_W4A8_STREAM
+    if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
+    return launch_status("gemv_w4a8");
+  }
+  const unsigned grid = (unsigned)((N + ck::w4a8::kRows - 1) / ck::w4a8::kRows);
   if (M <= 8)
     ck::w4a8::gemv_w4a8_kernel<1><<<grid, ck::w4a8::kWarps * 32, 0, S(stream)>>>(xq, x_scale, (int)M, (int)K, (int)N, w_packed, sw, bb, yy);
   else
@@ -516,6 +561,49 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
   if (!aligned(x, 16) || !aligned(qweight, 16)) return fail(CK_ERR_UNSUPPORTED, "gemv_awq_w4a16: x and qweight must be 16-byte aligned");
   if (!aligned(wscales, 2) || !aligned(wzeros, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "gemv_awq_w4a16: misaligned scales, zeros, bias or output");
+  if (K <= 4096 && K / group_size <= 256 && N % 8 == 0 && aligned(wscales, 16) && aligned(wzeros, 16)) {
+    // streaming path: 16-row weight tiles plus their scales and zeros through a shared-memory ring
+    using namespace ck::gstream;
+    CUtensorMap ts, tz;
+    const uint32_t ngrp = (uint32_t)(K / group_size);
+    ck_status r = make_tmap(&ts, wscales, (uint64_t)N, ngrp, (uint64_t)N * 2, 16, ngrp, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_DATA_TYPE_UINT16);
+    if (r != CK_OK) return r;
+    r = make_tmap(&tz, wzeros, (uint64_t)N, ngrp, (uint64_t)N * 2, 16, ngrp, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_DATA_TYPE_UINT16);
+    if (r != CK_OK) return r;
+    AwqParams ap;
+    ap.x = x; ap.qw = qweight; ap.bias = bias; ap.y = y;
+    ap.M = (int)M; ap.K = (int)K; ap.N = (int)N; ap.G = group_size;
+    ap.ntiles = (int)((N + 15) / 16);
+    ap.w_bytes = 16 * (int)(K / 2);
+    ap.sz_bytes = (int)ngrp * 16 * 2;
+    const int grid = std::min(ap.ntiles, sm_count());
+    const int tpc = (ap.ntiles + grid - 1) / grid;
+    ap.L = stream_layout(ap.w_bytes + 2 * ap.sz_bytes, 16 * tpc * 4 + 16);
+    const int nsub = (int)(K / 64), spw = (nsub + kCons - 1) / kCons;
+    cudaError_t e = cudaSuccess;
+#define CK_AWQ_STREAM(T, SPW)                                                                    \
+    {                                                                                            \
+      auto kern = awq_stream_kernel<T, SPW>;                                                     \
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ap.L.total);   \
+      if (e == cudaSuccess) kern<<<grid, kThreads, ap.L.total, S(stream)>>>(ts, tz, ap);         \
+    }
+    if (dt == CK_BF16) {
+      if (spw <= 2) CK_AWQ_STREAM(__nv_bfloat16, 2)
+      else if (spw <= 4) CK_AWQ_STREAM(__nv_bfloat16, 4)
+      else if (spw <= 6) CK_AWQ_STREAM(__nv_bfloat16, 6)
+      else CK_AWQ_STREAM(__nv_bfloat16, 8)
+    } else {
+      if (spw <= 2) CK_AWQ_STREAM(__half, 2)
+      else if (spw <= 4) CK_AWQ_STREAM(__half, 4)
+      else if (spw <= 6) CK_AWQ_STREAM(__half, 6)
+      else CK_AWQ_STREAM(__half, 8)
+    }
+#undef CK_AWQ_STREAM
+    if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_awq_w4a16: %s", cudaGetErrorString(e));
+    return launch_status("gemv_awq_w4a16");
+  }
   const unsigned grid = (unsigned)((N + ck::awq::kRows - 1) / ck::awq::kRows);
   if (dt == CK_BF16) {
     using T = __nv_bfloat16;

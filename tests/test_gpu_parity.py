@@ -347,6 +347,19 @@ def test_gemv_w4a8_ragged_bit_exact(ck, M, K, N, bias):
     np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
 
 
+@pytest.mark.parametrize("M,K,N", [(5, 8192, 96), (16, 4224, 40)])
+def test_gemv_w4a8_general_path_bit_exact(ck, M, K, N):
+    # K > 4096 takes the general (non-streaming) kernel
+    g = torch.Generator().manual_seed(K + N)
+    xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    xs = torch.rand(M, generator=g) * 0.1 + 0.001
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N,), 0.005, 0.02, g)
+    y = ck.gemv_w4a8(xq.to(DEV), xs.to(DEV), wp.to(DEV), sw.to(DEV))
+    r = O.gemv_w4a8(xq.numpy(), xs.numpy(), wp.numpy(), to_np_f64(sw))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
+
+
 def test_gemv_w4a8_agrees_with_large_m_gemm(ck):
     # the decode GEMV and the tensor-core GEMM share codec and epilogue: same int32 results
     g = torch.Generator().manual_seed(5)
@@ -373,9 +386,11 @@ def test_gemv_awq_config(ck, M):
 
 @pytest.mark.parametrize("M,K,N,G,dtype,bias", [
     (1, 128, 40, 64, torch.bfloat16, True),
-    (5, 1024, 70, 128, torch.float16, False),
-    (8, 768, 33, 256, torch.bfloat16, True),
+    (5, 1024, 70, 128, torch.float16, False),      # N % 8 != 0: general kernel
+    (8, 768, 33, 256, torch.bfloat16, True),       # general kernel
     (2, 3072, 96, 64, torch.float16, True),
+    (3, 8192, 48, 64, torch.bfloat16, True),       # K > 4096: general kernel
+    (4, 4096, 4104, 128, torch.bfloat16, False),   # ragged last 16-row tile
 ])
 def test_gemv_awq_variants(ck, M, K, N, G, dtype, bias):
     g = torch.Generator().manual_seed(K + N)
