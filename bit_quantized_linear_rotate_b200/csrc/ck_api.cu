@@ -576,11 +576,12 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
     ap.x = x; ap.qw = qweight; ap.bias = bias; ap.y = y;
     ap.M = (int)M; ap.K = (int)K; ap.N = (int)N; ap.G = group_size;
     ap.ntiles = (int)((N + 15) / 16);
-    ap.w_bytes = 16 * (int)(K / 2);
+    ap.w_bytes = 16 * (int)(K / 2);                   // a multiple of 512 (K % 64 == 0)
     ap.sz_bytes = (int)ngrp * 16 * 2;
+    ap.sz_stride = (ap.sz_bytes + 127) / 128 * 128;    // every tensor-copy destination 128-byte aligned
     const int grid = std::min(ap.ntiles, sm_count());
     const int tpc = (ap.ntiles + grid - 1) / grid;
-    ap.L = stream_layout(ap.w_bytes + 2 * ap.sz_bytes, 16 * tpc * 4 + 16);
+    ap.L = stream_layout(ap.w_bytes + 2 * ap.sz_stride, 16 * tpc * 4 + 16);
     const int nsub = (int)(K / 64), spw = (nsub + kCons - 1) / kCons;
     cudaError_t e = cudaSuccess;
 #define CK_AWQ_STREAM(T, SPW)                                                                    \

@@ -246,6 +246,7 @@ struct AwqParams {
   int ntiles;                    // 16-row weight tiles
   int w_bytes;                   // 16 * K / 2
   int sz_bytes;                  // (K / G) * 16 * 2: one of scales / zeros per stage
+  int sz_stride;                 // sz_bytes rounded up to 128: TMA destinations are 128-byte aligned
   Layout L;
 };
 
@@ -327,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&full[s], (i / ns) & 1, abort, 24)) break;
       const uint8_t* st = sm + s * L.stage_bytes;
       const T* sc = reinterpret_cast<const T*>(st + p.w_bytes);                 // [K/G][16]
-      const T* zr = reinterpret_cast<const T*>(st + p.w_bytes + p.sz_bytes);
+      const T* zr = reinterpret_cast<const T*>(st + p.w_bytes + p.sz_stride);
       float yacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int i2 = 0; i2 < SPW; ++i2) {
@@ -373,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[s], wb + 2u * (uint32_t)p.sz_bytes);
         bulk_load(st, p.qw + (int64_t)tile * 16 * wld, wb, &full[s]);
         tma_load_2d(st + p.w_bytes, &tm_s, &full[s], 16 * tile, 0);
-        tma_load_2d(st + p.w_bytes + p.sz_bytes, &tm_z, &full[s], 16 * tile, 0);
+        tma_load_2d(st + p.w_bytes + p.sz_stride, &tm_z, &full[s], 16 * tile, 0);
         issued = i + 1;
       }
       if (*abort)
