@@ -284,17 +284,40 @@ def time_linear_e2e(ck, w, steps: int, warmup: int, dev):
             "ms_per_step": ms}
 
 
-def time_rotating(fn, n_copies: int, iters: int, warmup: int):
+def time_rotating(fn, n_copies: int, iters: int, warmup: int, graph: bool = True):
+    """Device ms per call of fn(copy) over rotating buffer copies.
+
+    With graph=True the calls are captured once in a CUDA graph (as a decode
+    loop would run them) and the graph is replayed, so the timing is the
+    kernels' back-to-back device time rather than the host's launch rate.
+    """
     for i in range(warmup):
         fn(i % n_copies)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if not graph:
+        a.record()
+        for i in range(iters):
+            fn(i % n_copies)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+    per_graph = n_copies * max(1, 20 // n_copies)
+    cg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cg, capture_error_mode="relaxed"):
+        for i in range(per_graph):
+            fn(i % n_copies)
+    cg.replay()
+    torch.cuda.synchronize()
+    reps = max(1, iters // per_graph)
     a.record()
-    for i in range(iters):
-        fn(i % n_copies)
+    for _ in range(reps):
+        cg.replay()
     b.record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / iters
+    ms = a.elapsed_time(b) / (reps * per_graph)
+    del cg
+    return ms
 
 
 def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):

@@ -88,6 +88,20 @@ ck_status make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
   return CK_OK;
 }
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device
+// (cached per kernel instantiation through Tag; the largest value set wins).
+template <typename Tag, typename KernelT>
+cudaError_t set_smem_max(KernelT kern, int bytes) {
+  static int done[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
+  if (done[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
+  if (e == cudaSuccess) done[dev] = 200 * 1024 + 1024;
+  return e;
+}
+
 // Shared-memory layout of a streaming GEMV: as many stages as fit in ~200 KB.
 ck::gstream::Layout stream_layout(int stage_bytes, int misc_bytes) {
   using namespace ck::gstream;
@@ -528,7 +542,8 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
 #define CK_W4A8_STREAM(CPW)                                                                      \
     {                                                                                            \
       auto kern = w4a8_stream_kernel<CPW>;                                                       \
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sp.L.total);   \
+      struct Tag {};                                                                             \
+      e = set_smem_max<Tag>(kern, sp.L.total);                                                   \
       if (e == cudaSuccess) kern<<<grid, kThreads, sp.L.total, S(stream)>>>(sp);                 \
     }
     if (cpw <= 1) CK_W4A8_STREAM(1)
@@ -587,7 +602,8 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
 #define CK_AWQ_STREAM(T, SPW)                                                                    \
     {                                                                                            \
       auto kern = awq_stream_kernel<T, SPW>;                                                     \
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ap.L.total);   \
+      struct Tag {};                                                                             \
+      e = set_smem_max<Tag>(kern, ap.L.total);                                                   \
       if (e == cudaSuccess) kern<<<grid, kThreads, ap.L.total, S(stream)>>>(ts, tz, ap);         \
     }
     if (dt == CK_BF16) {
