@@ -536,7 +536,8 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
     sp.ntiles = (int)((N + 7) / 8);
     const int grid = std::min(sp.ntiles, sm_count());
     const int tpc = (sp.ntiles + grid - 1) / grid;
-    sp.L = stream_layout(8 * (int)(K / 2), kCons * 16 * 4 + 2 * 8 * tpc * 4 + 16);
+    sp.srow = (int)(K / 2) + 64;
+    sp.L = stream_layout(8 * sp.srow, kCons * 16 * 4 + 2 * 8 * tpc * 4 + 16);
     const int nchunk = (int)(K / 128), cpw = (nchunk + kCons - 1) / kCons;
     cudaError_t e;
 #define CK_W4A8_STREAM(CPW)                                                                      \
@@ -591,7 +592,8 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
     ap.x = x; ap.qw = qweight; ap.bias = bias; ap.y = y;
     ap.M = (int)M; ap.K = (int)K; ap.N = (int)N; ap.G = group_size;
     ap.ntiles = (int)((N + 15) / 16);
-    ap.w_bytes = 16 * (int)(K / 2);                   // a multiple of 512 (K % 64 == 0)
+    ap.srow = (int)(K / 2) + 32;
+    ap.w_bytes = (16 * ap.srow + 127) / 128 * 128;    // padded rows; the scale tiles follow 128-byte aligned
     ap.sz_bytes = (int)ngrp * 16 * 2;
     ap.sz_stride = (ap.sz_bytes + 127) / 128 * 128;    // every tensor-copy destination 128-byte aligned
     const int grid = std::min(ap.ntiles, sm_count());

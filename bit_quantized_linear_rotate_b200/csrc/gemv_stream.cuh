@@ -68,6 +68,7 @@ struct W4A8Params {
   __nv_bfloat16* y;              // (M, N)
   int M, K, N;
   int ntiles;                    // 8-row weight tiles
+  int srow;                      // shared-memory row stride: K/2 + 64 (bank-conflict-free reads)
   Layout L;
 };
 
@@ -92,7 +93,17 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_stream_kernel(const W4A8Para
   const int nchunk = p.K >> 7;
   const int ns = L.ns;
 
-  if (threadIdx.x == 0) {
+  // the producer initialises the barriers and starts streaming at once: the
+  // first ns tiles need no free-slot wait, so their copies overlap the prologue
+  auto issue = [&](int i) {
+    const int s = i % ns;
+    const int tile = t0 + i;
+    const int rows = min(8, p.N - 8 * tile);
+    mbar_arrive_expect_tx(&full[s], (uint32_t)(rows * wld));
+    for (int r = 0; r < rows; ++r)
+      bulk_load(sm + s * L.stage_bytes + r * p.srow, p.w + ((int64_t)tile * 8 + r) * wld, (uint32_t)wld, &full[s]);
+  };
+  if (warp == W_PROD && lane == 0) {
     for (int s = 0; s < ns; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&consumed[s], kCons);
@@ -100,6 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_stream_kernel(const W4A8Para
     }
     *abort_flag = 0;
     fence_mbarrier_init();
+    for (int i = 0; i < min(ns, nt); ++i) issue(i);
   }
 
   uint32_t af[CPW][4][4];
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_stream_kernel(const W4A8Para
       for (int ci = 0; ci < CPW; ++ci) {
         const int c = warp + kCons * ci;
         if (c < nchunk) {
-          const uint4 wv = *reinterpret_cast<const uint4*>(st + g * wld + c * 64 + 16 * t);
+          const uint4 wv = *reinterpret_cast<const uint4*>(st + g * p.srow + c * 64 + 16 * t);
           const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j)   // word j: k = 32t + 8j .. +7; low nibbles = even k
@@ -181,15 +193,10 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_stream_kernel(const W4A8Para
     }
   } else if (warp == W_PROD) {
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nt; ++i) {
-        const int s = i % ns;
-        if (!mbar_wait(&epi_done[s], ((i / ns) & 1) ^ 1, abort, 21)) break;
-        const int tile = t0 + i;
-        const int rows = min(8, p.N - 8 * tile);
-        const uint32_t bytes = (uint32_t)(rows * wld);
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_load(sm + s * L.stage_bytes, p.w + (int64_t)tile * 8 * wld, bytes, &full[s]);
+      int issued = min(ns, nt);
+      for (int i = issued; i < nt; ++i) {
+        if (!mbar_wait(&epi_done[i % ns], ((i / ns) & 1) ^ 1, abort, 21)) break;
+        issue(i);
         issued = i + 1;
       }
       if (*abort)
@@ -247,6 +254,7 @@ struct AwqParams {
   int w_bytes;                   // 16 * K / 2
   int sz_bytes;                  // (K / G) * 16 * 2: one of scales / zeros per stage
   int sz_stride;                 // sz_bytes rounded up to 128: TMA destinations are 128-byte aligned
+  int srow;                      // shared-memory row stride: K/2 + 32 (bank-conflict-free reads)
   Layout L;
 };
 
@@ -274,7 +282,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ns = L.ns;
   const T* x = reinterpret_cast<const T*>(p.x);
 
-  if (threadIdx.x == 0) {
+  // the producer initialises the barriers and starts streaming at once (see the W4A8 kernel)
+  auto issue = [&](int i) {
+    const int s = i % ns;
+    const int tile = t0 + i;
+    const int rows = min(16, p.N - 16 * tile);
+    uint8_t* st = sm + s * L.stage_bytes;
+    mbar_arrive_expect_tx(&full[s], (uint32_t)(rows * wld) + 2u * (uint32_t)p.sz_bytes);
+    for (int r = 0; r < rows; ++r)
+      bulk_load(st + r * p.srow, p.qw + ((int64_t)tile * 16 + r) * wld, (uint32_t)wld, &full[s]);
+    tma_load_2d(st + p.w_bytes, &tm_s, &full[s], 16 * tile, 0);
+    tma_load_2d(st + p.w_bytes + p.sz_stride, &tm_z, &full[s], 16 * tile, 0);
+  };
+  if (warp == W_PROD && lane == 0) {
+    prefetch_tmap(&tm_s);
+    prefetch_tmap(&tm_z);
     for (int s = 0; s < ns; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&consumed[s], kCons);
@@ -282,10 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     *abort_flag = 0;
     fence_mbarrier_init();
-  }
-  if (warp == W_PROD && lane == 0) {
-    prefetch_tmap(&tm_s);
-    prefetch_tmap(&tm_z);
+    for (int i = 0; i < min(ns, nt); ++i) issue(i);
   }
 
   uint32_t bp[SPW][8];    // activation fragments (token g, k = sb*64 + 16t + (k, k+4) pairs)
@@ -334,8 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i2 = 0; i2 < SPW; ++i2) {
         const int sb = warp + kCons * i2;
         if (sb < nsub) {
-          const uint2 w0 = *reinterpret_cast<const uint2*>(st + g * wld + sb * 32 + 8 * t);
-          const uint2 w1 = *reinterpret_cast<const uint2*>(st + (g + 8) * wld + sb * 32 + 8 * t);
+          const uint2 w0 = *reinterpret_cast<const uint2*>(st + g * p.srow + sb * 32 + 8 * t);
+          const uint2 w1 = *reinterpret_cast<const uint2*>(st + (g + 8) * p.srow + sb * 32 + 8 * t);
           const uint32_t r0[2] = {w0.x, w0.y}, r1[2] = {w1.x, w1.y};
           float P[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -363,18 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == W_PROD) {
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nt; ++i) {
-        const int s = i % ns;
-        if (!mbar_wait(&epi_done[s], ((i / ns) & 1) ^ 1, abort, 25)) break;
-        const int tile = t0 + i;
-        const int rows = min(16, p.N - 16 * tile);
-        const uint32_t wb = (uint32_t)(rows * wld);
-        uint8_t* st = sm + s * L.stage_bytes;
-        mbar_arrive_expect_tx(&full[s], wb + 2u * (uint32_t)p.sz_bytes);
-        bulk_load(st, p.qw + (int64_t)tile * 16 * wld, wb, &full[s]);
-        tma_load_2d(st + p.w_bytes, &tm_s, &full[s], 16 * tile, 0);
-        tma_load_2d(st + p.w_bytes + p.sz_stride, &tm_z, &full[s], 16 * tile, 0);
+      int issued = min(ns, nt);
+      for (int i = issued; i < nt; ++i) {
+        if (!mbar_wait(&epi_done[i % ns], ((i / ns) & 1) ^ 1, abort, 25)) break;
+        issue(i);
         issued = i + 1;
       }
       if (*abort)
