@@ -168,7 +168,7 @@ template <int QBITS, int STORE, int GT, typename T>
 void launch_rq_g(const T* x, int64_t M, int K, int64_t ldx, int G, float rnorm, uint8_t* q, float* s, int32_t* rs,
                  int nt, cudaStream_t st) {
   auto kern = ck::rq::rotate_quant_kernel<QBITS, STORE, GT, T>;
-  const size_t smem = (size_t)(nt / 32) * 2048;     // one 2 KB transpose buffer per warp
+  const size_t smem = (size_t)(nt / 32) * 32 * ck::rq::CPT * 16;   // one transpose buffer per warp
   struct Tag {};
   kern<<<persistent_grid<Tag>(kern, nt, smem, M), nt, smem, st>>>(x, M, K, ldx, G, rnorm, q, s, rs);
 }
@@ -204,7 +204,7 @@ ck_status rotate_quant_impl(const void* x, ck_dtype xt, int64_t M, int64_t K, in
                             int bits, int store, void* q, float* s, int32_t* rs, cudaStream_t st) {
   using namespace ck::rq;
   const int64_t nt = ((K + EPT - 1) / EPT + 31) / 32 * 32;
-  if (nt > 1024) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K=%lld too large (max 32768)", (long long)K);
+  if (nt > 512) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K=%lld too large (max 32768)", (long long)K);
   if (xt == CK_BF16) launch_rq_store<__nv_bfloat16>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, st);
   else launch_rq_store<__half>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, st);
   return launch_status("rotate_quant");

@@ -7,9 +7,10 @@
 // named by comfy-kitchen PR #182 ("Description").
 //
 // A persistent grid of CTAs walks the rows, one row per CTA at a time, the next
-// row's loads issued before the current row is processed; thread t owns the 32
-// contiguous columns [32t, 32t + 32) (four 128-bit loads). The transform runs in fp32: log2(min(G, 32)) butterfly
-// stages inside the thread, then log2(G / 32) stages across lanes
+// row's loads issued before the current row is processed; thread t owns the 64
+// contiguous columns [64t, 64t + 64) (eight 128-bit loads, issued coalesced and
+// regrouped through shared memory). The transform runs in fp32: log2(min(G, 64)) butterfly
+// stages inside the thread, then log2(G / 64) stages across lanes
 // (__shfl_xor_sync, one shuffle and one FMA per element and stage), then the
 // 1/sqrt(G) normalisation (a power of two for G = 16, 64, 256). The rotated row
 // never leaves registers: amax is reduced across the CTA, then every thread
@@ -31,7 +32,8 @@
 namespace ck {
 namespace rq {
 
-constexpr int EPT = 32;   // columns per thread
+constexpr int EPT = 64;   // columns per thread
+constexpr int CPT = EPT / 8;   // 16-byte chunks per thread
 
 // STORE_INT8_PERM: int8 codes with the columns of each 8-column group stored in
 // the order (0 2 4 6 1 3 5 7), plus the row sum of the codes -- the activation
@@ -39,29 +41,29 @@ constexpr int EPT = 32;   // columns per thread
 // nibbles without byte shuffles).
 enum Store { STORE_PACKED4 = 0, STORE_INT8 = 1, STORE_INT8_PERM = 2 };
 
-// Coalesced 128-bit loads of the warp's 1024 columns: lane l takes 16-byte
-// chunks l, 32 + l, 64 + l, 96 + l of the warp's span (zero past K).
-__device__ __forceinline__ void load_raw(const void* row, int warp, int lane, int K, uint4 (&raw)[EPT / 8]) {
+// Coalesced 128-bit loads of the warp's 32 * EPT columns: lane l takes 16-byte
+// chunks l, 32 + l, ... of the warp's span (zero past K).
+__device__ __forceinline__ void load_raw(const void* row, int warp, int lane, int K, uint4 (&raw)[CPT]) {
 #pragma unroll
-  for (int j = 0; j < EPT / 8; ++j) {
-    const int c = 128 * warp + 32 * j + lane;           // 16-byte chunk index in the row
+  for (int j = 0; j < CPT; ++j) {
+    const int c = 32 * CPT * warp + 32 * j + lane;      // 16-byte chunk index in the row
     raw[j] = (8 * c < K) ? __ldcs(reinterpret_cast<const uint4*>(row) + c) : make_uint4(0, 0, 0, 0);
   }
 }
 
-// 16-byte slot of chunk c in a warp's 2 KB transpose buffer: the low three bits
+// 16-byte slot of chunk c in a warp's transpose buffer: the low three bits
 // (position in a 128-byte line) are XORed with the line index, so both the
 // coalesced writes and the contiguous per-thread reads are bank-conflict free.
 __device__ __forceinline__ int tslot(int c) { return c ^ ((c >> 3) & 7); }
 
-// Regroups the coalesced chunks so that lane l holds chunks 4l .. 4l + 3 (its
-// 32 contiguous columns).
-__device__ __forceinline__ void transpose_raw(uint4* buf, int lane, uint4 (&raw)[EPT / 8]) {
+// Regroups the coalesced chunks so that lane l holds chunks CPT*l .. CPT*l + CPT-1
+// (its EPT contiguous columns).
+__device__ __forceinline__ void transpose_raw(uint4* buf, int lane, uint4 (&raw)[CPT]) {
 #pragma unroll
-  for (int j = 0; j < EPT / 8; ++j) buf[tslot(32 * j + lane)] = raw[j];
+  for (int j = 0; j < CPT; ++j) buf[tslot(32 * j + lane)] = raw[j];
   __syncwarp();
 #pragma unroll
-  for (int j = 0; j < EPT / 8; ++j) raw[j] = buf[tslot(4 * lane + j)];
+  for (int j = 0; j < CPT; ++j) raw[j] = buf[tslot(CPT * lane + j)];
   __syncwarp();
 }
 
@@ -127,7 +129,7 @@ __device__ __forceinline__ void fht_in_thread(float2 (&v)[EPT / 2], int G) {
   }
 }
 
-// Index bits 5.. live in lane bits 0..: new = partner + v (bit clear) or partner - v (bit set).
+// Index bits log2(EPT).. live in lane bits 0..: new = partner + v (bit clear) or partner - v (bit set).
 __device__ __forceinline__ void fht_across_lanes(float2 (&v)[EPT / 2], int G, int lane) {
   for (int j = 1; EPT * j < G; j <<= 1) {
     const float sg = (lane & j) ? -1.0f : 1.0f;
@@ -161,37 +163,40 @@ __device__ __forceinline__ float quant_exact(float y, float r, float s) {
 // GT: the group size when it is 1, 16, 64 or 256 (compile time), 0 otherwise
 // (then taken from G at run time).
 template <int QBITS, int STORE, int GT, typename T>
-__global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
+__global__ void __launch_bounds__(512) rotate_quant_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
                                                             int G_rt, float rnorm, uint8_t* __restrict__ q,
                                                             float* __restrict__ scale,
                                                             int32_t* __restrict__ rowsum) {
   constexpr float kQmax = QBITS == 4 ? 7.0f : 127.0f;
   const int G = GT ? GT : G_rt;
   __shared__ float red[4][32];   // [2 * (it & 1)]: amax, [2 * (it & 1) + 1]: row sum
-  extern __shared__ uint4 tbuf_all[];              // 2 KB per warp
+  extern __shared__ uint4 tbuf_all[];              // 32 * CPT chunks per warp
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int e0 = tid * EPT;
-  uint4* tbuf = tbuf_all + 128 * warp;
+  uint4* tbuf = tbuf_all + 32 * CPT * warp;
 
-  // persistent over rows; the next row's 128-bit loads are in flight while
-  // the current row is transformed, reduced and quantized
+  // persistent over rows; the next row's 128-bit loads are in flight while the
+  // current row is transformed, reduced and quantized (not for G = 256 or a
+  // run-time G, whose cross-lane stages need those registers)
+  constexpr bool kPrefetch = GT != 0 && GT <= EPT;
   int64_t row = blockIdx.x;
-  uint4 raw[EPT / 8];
-  if (row < M) load_raw(x + row * ldx, warp, lane, K, raw);
+  uint4 raw[CPT];
+  if (kPrefetch && row < M) load_raw(x + row * ldx, warp, lane, K, raw);
   for (int it = 0; row < M; row += gridDim.x, ++it) {
+    if (!kPrefetch) load_raw(x + row * ldx, warp, lane, K, raw);
     transpose_raw(tbuf, lane, raw);
     float2 v[EPT / 2];
 #pragma unroll
-    for (int j = 0; j < EPT / 8; ++j) {
+    for (int j = 0; j < CPT; ++j) {
       float f[8];
       to_float8<T>(raw[j], f);
 #pragma unroll
       for (int e = 0; e < 4; ++e) v[4 * j + e] = make_float2(f[2 * e], f[2 * e + 1]);
     }
     const int64_t next = row + gridDim.x;
-    if (next < M) load_raw(x + next * ldx, warp, lane, K, raw);
+    if (kPrefetch && next < M) load_raw(x + next * ldx, warp, lane, K, raw);
 
     // unnormalised transform z = x H; the 1/sqrt(G) factor is folded into the scale
     fht_in_thread(v, G);
@@ -264,28 +269,31 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const T* __restrict_
     if (e0 < K) {
       if (STORE == STORE_PACKED4) {
         // bytes hold u = q + 8 < 16: fold neighbours into nibbles, low nibble = even column
-        uint32_t w[4];
+        uint32_t w[EPT / 8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < EPT / 8; ++j) {
           const uint32_t ta = g[2 * j] | (g[2 * j] >> 4), tb = g[2 * j + 1] | (g[2 * j + 1] >> 4);
           w[j] = __byte_perm(ta, tb, 0x6420);
         }
         uint8_t* qr = q + row * (int64_t)(K >> 1) + (e0 >> 1);
-        if ((K & 31) == 0) {          // rows of K/2 bytes are 16-byte aligned
-          *reinterpret_cast<uint4*>(qr) = make_uint4(w[0], w[1], w[2], w[3]);
+        if ((K & 31) == 0 && e0 + EPT <= K) {          // whole, 16-byte aligned pieces
+#pragma unroll
+          for (int j = 0; j < EPT / 32; ++j)
+            reinterpret_cast<uint4*>(qr)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < EPT / 8; ++j)
             if (e0 + 8 * j < K) reinterpret_cast<uint32_t*>(qr)[j] = w[j];
         }
       } else {
         uint8_t* qr = q + row * (int64_t)K + e0;
-        if ((K & 31) == 0) {
-          reinterpret_cast<uint4*>(qr)[0] = make_uint4(g[0], g[1], g[2], g[3]);
-          reinterpret_cast<uint4*>(qr)[1] = make_uint4(g[4], g[5], g[6], g[7]);
+        if ((K & 31) == 0 && e0 + EPT <= K) {
+#pragma unroll
+          for (int j = 0; j < EPT / 16; ++j)
+            reinterpret_cast<uint4*>(qr)[j] = make_uint4(g[4 * j], g[4 * j + 1], g[4 * j + 2], g[4 * j + 3]);
         } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < EPT / 8; ++j)
             if (e0 + 8 * j < K) reinterpret_cast<uint2*>(qr)[j] = make_uint2(g[2 * j], g[2 * j + 1]);
         }
       }
