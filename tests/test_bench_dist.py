@@ -1,0 +1,76 @@
+"""Host logic of bench.py for N > 1 ranks, on CPU with gloo at world size 2.
+
+The path shards as independent replicas, so the only cross-rank steps are the
+barrier around the timed region and the max over ranks of the timed
+duration; the reference arm runs on rank 0 alone.
+"""
+
+import contextlib
+import io
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, q):
+    os.environ.update(WORLD_SIZE=str(world), RANK=str(rank), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch.distributed as dist
+    try:
+        w, r, _ = bench.dist_setup()
+        assert (w, r) == (world, rank)
+        assert dist.get_backend() == "gloo"
+        bench.barrier(w)
+        # each rank "measured" a different duration: everyone must see the slowest
+        slowest = bench.max_over_ranks(10.0 + rank, w)
+        # the reference arm prints one line on rank 0 and nothing elsewhere
+        out = io.StringIO()
+        with contextlib.redirect_stdout(out):
+            if rank != 0:
+                bench.run_reference(type("A", (), {"warmup": 0, "steps": 1, "cpu_rows": 1})(), w, rank)
+        q.put((rank, slowest, out.getvalue()))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def test_two_rank_barrier_and_max_over_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+            pytest.fail("rank did not finish")
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    assert [g[1] for g in got] == [11.0, 11.0]
+    assert got[1][2] == ""          # rank 1 printed nothing
+
+
+def test_value_is_aggregate_units_over_slowest_rank():
+    # value = 2*M*N*K*steps*world / slowest time, i.e. per-rank work is fixed (weak scaling)
+    sys.path.insert(0, ROOT)
+    import bench  # noqa: F401
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    assert "ops * world / (ms_step * 1e-3)" in src
+    assert "max_over_ranks(t[\"total_ms\"], world)" in src
