@@ -46,6 +46,7 @@ SIGNATURES = {
     "ck_linear_w4a4": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
     "ck_linear_w4a4_quantize": [_p, _int, _i64, _i64, _i64, _int, _p, ctypes.c_size_t, _p],
     "ck_linear_w4a4_matmul": [_i64, _i64, _i64, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
+    "ck_linear_w4a4_static": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "ck_gemv_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemv_awq_w4a16": [_p, _int, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p],
     "ck_gemm_w4a4_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
@@ -225,6 +226,27 @@ def linear_w4a4(x, w_packed, w_scale, group_size: int, bias=None, workspace=None
                               _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)),
            "ck_linear_w4a4")
+    return out
+
+
+# Size of the library's built-in scratch for linear_w4a4_static (CK_LINEAR_STATIC_SCRATCH_BYTES).
+LINEAR_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def linear_w4a4_static(x, w_packed, w_scale, group_size: int, bias=None, out=None, stream=None):
+    """linear_w4a4 without a workspace argument: the library uses its own fixed per-device scratch.
+
+    Same results as linear_w4a4. Calls on one device share that scratch, so calls that may run
+    at the same time on the GPU (different streams, several threads) must not be mixed.
+    """
+    _cuda(x, w_packed, w_scale, bias)
+    M, K, ldx, x2 = _rows(x)
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), device=x.device, dtype=torch.bfloat16)
+    _check(lib.ck_linear_w4a4_static(_ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size, _ptr(w_packed),
+                                     _ptr(w_scale), _ptr(bias), _ptr(out), _stream(stream)),
+           "ck_linear_w4a4_static")
     return out
 
 

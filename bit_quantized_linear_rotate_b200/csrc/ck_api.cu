@@ -493,6 +493,65 @@ ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64
   return ck_linear_w4a4_matmul(M, K, N, w_packed, w_scale, bias, y, workspace, ws_bytes, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------- linear with a static scratch
+
+// The scratch of ck_linear_w4a4_static: one fixed block of global memory per
+// device, reserved when the module loads on that device. It holds the same
+// layout as the caller workspace of ck_linear_w4a4 (codes, scales, row sums).
+static __device__ __align__(256) unsigned char g_linear_scratch[CK_LINEAR_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_linear_scratch on the current device, looked up on the
+// first call for that device and cached.
+ck_status static_scratch_addr(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess)
+    return fail(CK_ERR_CUDA, "linear_w4a4_static: cudaGetDevice failed: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxScratchDevices)
+    return fail(CK_ERR_UNSUPPORTED, "linear_w4a4_static: device ordinal %d >= %d", dev, kMaxScratchDevices);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_linear_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(CK_ERR_CUDA, "linear_w4a4_static: cudaGetSymbolAddress failed on device %d: %s", dev,
+                  cudaGetErrorString(e));
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return CK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ck_status ck_linear_w4a4_static(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N,
+                                int64_t ldx, int group_size, const uint8_t* w_packed,
+                                const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                                void* stream) {
+  ck_status r = check_gemm_shape("linear_w4a4_static", M, K, N);
+  if (r != CK_OK) return r;
+  const size_t need = linear_ws_bytes(M, K);
+  if (need > (size_t)CK_LINEAR_STATIC_SCRATCH_BYTES)
+    return fail(CK_ERR_UNSUPPORTED,
+                "linear_w4a4_static: M=%lld, K=%lld need %zu bytes of scratch, more than the %zu-byte "
+                "static scratch; call ck_linear_w4a4 with a workspace instead",
+                (long long)M, (long long)K, need, (size_t)CK_LINEAR_STATIC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if ((r = static_scratch_addr(&scratch)) != CK_OK) return r;
+  return ck_linear_w4a4(x, xt, M, K, N, ldx, group_size, w_packed, w_scale, bias, y, scratch,
+                        (size_t)CK_LINEAR_STATIC_SCRATCH_BYTES, stream);
+}
+
 ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, int64_t M, int64_t K,
                            int64_t N, int32_t* acc, void* stream) {
   ck_status r = check_gemm_shape("gemm_w4a4_i32", M, K, N);

@@ -167,6 +167,48 @@ ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* 
                                 const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
                                 const void* workspace, size_t ws_bytes, void* stream);
 
+/* Size of the scratch built into the library for ck_linear_w4a4_static: 32 MiB per device. */
+#define CK_LINEAR_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * ck_linear_w4a4 for callers that cannot hand the library a workspace. The
+ * ConvRot pages have no counterpart to this entry point; it exists only
+ * because of how some callers are built.
+ *
+ * Who needs it: a caller that owns the input and output buffers but has no
+ * way to get device scratch -- for example a plugin whose host passes it
+ * only tensors, or code running where cudaMalloc is not allowed because it
+ * can block or synchronise the device, or where every byte of device memory
+ * belongs to another allocator. Such a caller cannot use ck_linear_w4a4,
+ * which needs a workspace of ck_linear_w4a4_workspace_bytes(M, K) bytes.
+ *
+ * What it does: the same computation as ck_linear_w4a4 with the same
+ * arguments minus workspace/ws_bytes, and the same results bit for bit. The
+ * scratch is a fixed CK_LINEAR_STATIC_SCRATCH_BYTES block of device memory
+ * inside the library, reserved by the CUDA runtime when the library's GPU
+ * code is loaded on a device. The call allocates and frees nothing.
+ *
+ * Limits and rules:
+ * - The scratch must hold ck_linear_w4a4_workspace_bytes(M, K) bytes, i.e.
+ *   about M*K + 8*M. Larger problems (for instance M = 8192, K = 10240) get
+ *   CK_ERR_UNSUPPORTED with a message naming the sizes, and nothing runs.
+ *   M = 8192, K = 3840 fits.
+ * - Set-up: the first call on each device (with that device current) looks up
+ *   the scratch's device address and caches it. Make that first call before
+ *   starting any stream capture.
+ * - Nothing in the scratch needs to start at zero: every byte the GEMM phase
+ *   reads is written earlier in the same call by the quantize phase.
+ * - There is one scratch per device, shared by every call on that device.
+ *   Calls whose work can overlap on the GPU -- issued on different streams
+ *   without ordering between them, or from several host threads -- race on
+ *   it and may produce wrong results. Calls on one stream run one after
+ *   another and are safe.
+ */
+ck_status ck_linear_w4a4_static(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N,
+                                int64_t ldx, int group_size, const uint8_t* w_packed,
+                                const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                                void* stream);
+
 /*
  * W4A8 decode GEMV ("W4A8 decode GEMV" of comfy-kitchen PR #182, Description;
  * "asym_w4a8_int8" of stable-diffusion.cpp PR #2276): int8 activations times
