@@ -185,11 +185,16 @@ def oracle_linear_sample(w, rows: int):
     return dt
 
 
-def cpu_baseline(w, rows: int):
-    dt = oracle_linear_sample(w, rows)
-    ops = 2.0 * rows * w.N * w.K
-    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {rows} of {w.M} rows of {w.name} (full K, N), one pass, {dt:.2f} s"}
+def cpu_baseline(w, rows: int, min_seconds: float = 10.0, max_passes: int = 8):
+    """The oracle on `rows` rows of the workload, repeated until about `min_seconds` of CPU work."""
+    rows = min(rows, w.M)
+    total, passes = 0.0, 0
+    while passes < max_passes and (passes == 0 or total < min_seconds):
+        total += oracle_linear_sample(w, rows)
+        passes += 1
+    ops = 2.0 * rows * w.N * w.K * passes
+    return {"value": ops / total / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {rows} of {w.M} rows of {w.name} (full K, N), {passes} passes, {total:.1f} s"}
 
 
 # ------------------------------------------------------------------ GPU legs
@@ -335,7 +340,8 @@ def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
         allb = wbytes + 2 * w.N + M * w.K + 4 * M + 2 * M * w.N
         out[f"w4a8_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
                              "all_GBps": allb / (ms * 1e-3) / 1e9,
-                             "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R}
+                             "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R,
+                             "traffic": load_traffic("w4a8_stream_kernel") if M == 16 else None}
     w = WL.GEMV_AWQ
     for M in w.Ms:
         d = WL.gemv_awq_inputs(w, M)
@@ -352,7 +358,8 @@ def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
         allb = per + 2 * M * w.K + 2 * M * w.N
         out[f"awq_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
                             "all_GBps": allb / (ms * 1e-3) / 1e9,
-                            "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R}
+                            "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R,
+                            "traffic": load_traffic("awq_stream_kernel") if M == 4 else None}
     return out
 
 
@@ -408,11 +415,15 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     w = WL.LINEAR_M8192
+    # size each step's row sample so that the whole run stays around a minute of CPU time
+    probe_rows = 64
+    per_row = oracle_linear_sample(w, probe_rows) / probe_rows
+    rows = int(max(16, min(args.cpu_rows, 60.0 / max(1, args.steps + args.warmup) / per_row)))
     for _ in range(args.warmup):
-        oracle_linear_sample(w, min(args.cpu_rows, 16))
-    times = [oracle_linear_sample(w, args.cpu_rows) for _ in range(args.steps)]
+        oracle_linear_sample(w, rows)
+    times = [oracle_linear_sample(w, rows) for _ in range(args.steps)]
     dt = sum(times)
-    ops = 2.0 * args.cpu_rows * w.N * w.K * args.steps
+    ops = 2.0 * rows * w.N * w.K * args.steps
     v = ops / dt / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
@@ -421,7 +432,7 @@ def run_reference(args, world, rank):
             "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "G": w.G,
                        "step": "CPU oracle linear_w4a4 on a bounded row sample"},
             "cpu_baseline": {"value": v, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"first {args.cpu_rows} of {w.M} rows per step"},
+                             "sample": f"first {rows} of {w.M} rows per step"},
             "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -432,7 +443,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-rows", type=int, default=512, help="rows of the CPU oracle sample")
+    ap.add_argument("--cpu-rows", type=int, default=8192, help="rows of the CPU oracle sample (at most M)")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-siblings", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
