@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/ck.h"
 #include "ck_common.cuh"
@@ -49,6 +50,25 @@ ck_status launch_status(const char* what) {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Launches `kern` on `st` as a programmatic dependent of the previous kernel in
+// the stream: it may start while that kernel finishes and orders itself after
+// it with grid_dep_wait (ck_common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------- tensor maps
 
@@ -88,6 +108,10 @@ ck_status make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
   return CK_OK;
 }
 
+// Dynamic shared memory of one streaming-GEMV CTA: two CTAs (plus the 1 KB
+// the runtime reserves per CTA) fit in an SM's 228 KB.
+constexpr int kStreamSmemMax = 112 * 1024;
+
 // Raises a kernel's dynamic shared-memory limit to `bytes` once per device
 // (cached per kernel instantiation through Tag; the largest value set wins).
 template <typename Tag, typename KernelT>
@@ -97,18 +121,20 @@ cudaError_t set_smem_max(KernelT kern, int bytes) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
   if (done[dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
-  if (e == cudaSuccess) done[dev] = 200 * 1024 + 1024;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
+  if (e == cudaSuccess) done[dev] = kStreamSmemMax;
   return e;
 }
 
-// Shared-memory layout of a streaming GEMV: as many stages as fit in ~200 KB.
+// Shared-memory layout of a streaming GEMV: as many stages as fit in half of
+// an SM's shared memory, so that the next call's CTA can be resident (and
+// streaming its first tiles) while this one runs.
 ck::gstream::Layout stream_layout(int stage_bytes, int misc_bytes) {
   using namespace ck::gstream;
   Layout L;
   L.stage_bytes = (stage_bytes + 127) / 128 * 128;
   const int red_stage = kCons * 32 * 4 * 4;
-  const int budget = 200 * 1024 - misc_bytes - 3 * kMaxStages * 8 - 256;
+  const int budget = kStreamSmemMax - misc_bytes - 3 * kMaxStages * 8 - 256;
   L.ns = std::min(kMaxStages, budget / (L.stage_bytes + red_stage));
   L.off_red = L.ns * L.stage_bytes;
   L.off_misc = L.off_red + L.ns * red_stage;
@@ -170,7 +196,7 @@ void launch_rq_g(const T* x, int64_t M, int K, int64_t ldx, int G, float rnorm, 
   auto kern = ck::rq::rotate_quant_kernel<QBITS, STORE, GT, T>;
   const size_t smem = (size_t)(nt / 32) * 32 * ck::rq::CPT * 16;   // one transpose buffer per warp
   struct Tag {};
-  kern<<<persistent_grid<Tag>(kern, nt, smem, M), nt, smem, st>>>(x, M, K, ldx, G, rnorm, q, s, rs);
+  launch_pdl(kern, dim3(persistent_grid<Tag>(kern, nt, smem, M)), dim3(nt), smem, st, x, M, K, ldx, G, rnorm, q, s, rs);
 }
 
 template <int QBITS, int STORE, typename T>
@@ -282,17 +308,19 @@ ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const void*
   const int pairs = (int)std::min<int64_t>(tiles, pairs_max);
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
   if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemm_w4: launch failed: %s", cudaGetErrorString(e));
   return launch_status("gemm_w4");
@@ -604,7 +632,7 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
       auto kern = w4a8_stream_kernel<CPW>;                                                       \
       struct Tag {};                                                                             \
       e = set_smem_max<Tag>(kern, sp.L.total);                                                   \
-      if (e == cudaSuccess) kern<<<grid, kThreads, sp.L.total, S(stream)>>>(sp);                 \
+      if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), sp.L.total, S(stream), sp); \
     }
     if (cpw <= 1) CK_W4A8_STREAM(1)
     else if (cpw == 2) CK_W4A8_STREAM(2)
@@ -665,7 +693,7 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
       auto kern = awq_stream_kernel<T, SPW>;                                                     \
       struct Tag {};                                                                             \
       e = set_smem_max<Tag>(kern, ap.L.total);                                                   \
-      if (e == cudaSuccess) kern<<<grid, kThreads, ap.L.total, S(stream)>>>(ts, tz, ap);         \
+      if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), ap.L.total, S(stream), ts, tz, ap); \
     }
     if (dt == CK_BF16) {
       if (spw <= 2) CK_AWQ_STREAM(__nv_bfloat16, 2)

@@ -150,6 +150,18 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------ programmatic dependent launch
+
+// Kernels launched with the programmatic-stream-serialisation attribute may
+// start before the previous kernel in the stream has finished. grid_dep_wait
+// blocks until every grid this one depends on has completed and its memory
+// writes are visible: it must come before any read of data a previous kernel
+// produces and before any write. grid_dep_launch lets the next such kernel be
+// scheduled once every CTA of this grid has issued it (or exited). Both are
+// no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // --------------------------------------------------------------------- TMA
 
 // 2-D tiled TMA load (no multicast): box at coordinates (x = inner, y = row).

@@ -201,6 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort = abort_flag;
+  // launched as a programmatic dependent: the set-up above overlaps the end of
+  // the previous kernel; the operands and the output belong to it until here
+  grid_dep_launch();
+  grid_dep_wait();
 
   if (warp == W_PACK) {
     // ------------------------------------------------------ packed-tile producer

@@ -14,6 +14,15 @@
 //              applies the scales and writes y.
 // All barrier waits are bounded; a timeout sets the device error word.
 //
+// Back-to-back calls overlap: a CTA takes at most half of an SM's shared
+// memory, the kernels are launched as programmatic dependents, each lets the
+// next one be scheduled as soon as it starts, and a new call streams its first
+// weight tiles (constant data) into its ring while the previous call is still
+// running; only the activation reads and the output writes wait for the
+// previous kernel (grid_dep_wait). A decode loop of GEMVs thus keeps HBM
+// streaming across kernel boundaries instead of paying each launch's ramp-up
+// and drain.
+//
 // W4A8 (comfy-kitchen PR #182, "Description": register-side int4 decode, int32
 // accumulation, EpiRowwise): weights are the n8 operand of
 // mma.m16n8k32.s8.u8 (8 weight rows per tile), the <= 16 activation rows the
@@ -73,7 +82,7 @@ struct W4A8Params {
 };
 
 template <int CPW>   // 128-column chunks per consumer warp (K <= 8 * 128 * CPW)
-__global__ void __launch_bounds__(kThreads, 1) w4a8_stream_kernel(const W4A8Params p) {
+__global__ void __launch_bounds__(kThreads, 2) w4a8_stream_kernel(const W4A8Params p) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const Layout& L = p.L;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.off_bar);
@@ -113,6 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_stream_kernel(const W4A8Para
     fence_mbarrier_init();
     for (int i = 0; i < min(ns, nt); ++i) issue(i);
   }
+  grid_dep_launch();
+  grid_dep_wait();   // the activations and the output belong to the previous kernel until here
 
   uint32_t af[CPW][4][4];
   if (warp < kCons) {
@@ -259,7 +270,7 @@ struct AwqParams {
 };
 
 template <typename T, int SPW>   // 64-column sub-blocks per consumer warp (K <= 8 * 64 * SPW)
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     awq_stream_kernel(const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
                       const AwqParams p) {
   using Tr = awq::Traits<T>;
@@ -306,6 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbarrier_init();
     for (int i = 0; i < min(ns, nt); ++i) issue(i);
   }
+  grid_dep_launch();
+  grid_dep_wait();   // the activations and the output belong to the previous kernel until here
 
   uint32_t bp[SPW][8];    // activation fragments (token g, k = sb*64 + 16t + (k, k+4) pairs)
   float X[SPW][2];        // sum_k x for tokens 2t, 2t + 1 over each sub-block

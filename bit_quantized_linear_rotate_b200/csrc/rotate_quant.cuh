@@ -181,6 +181,10 @@ __global__ void __launch_bounds__(512) rotate_quant_kernel(const T* __restrict__
   // current row is transformed, reduced and quantized (not for G = 256 or a
   // run-time G, whose cross-lane stages need those registers)
   constexpr bool kPrefetch = GT != 0 && GT <= EPT;
+  // launched as a programmatic dependent: x and the outputs belong to the
+  // previous kernel in the stream until grid_dep_wait returns
+  grid_dep_launch();
+  grid_dep_wait();
   int64_t row = blockIdx.x;
   uint4 raw[CPT];
   if (kPrefetch && row < M) load_raw(x + row * ldx, warp, lane, K, raw);
