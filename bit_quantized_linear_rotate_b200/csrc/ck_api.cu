@@ -108,6 +108,28 @@ ck_status make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
   return CK_OK;
 }
 
+// 3-D tensor map over a packed weight matrix (N rows of K/2 bytes) viewed as
+// [K/128 slices of 64 bytes][N rows][64 bytes], slices outermost, with the
+// 64-byte swizzle; one box is `rows` rows x all slices (the streaming GEMVs'
+// tile layout, gemv_stream.cuh).
+ck_status make_tmap_wtile(CUtensorMap* m, const void* w, uint64_t N, uint64_t K, uint32_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(CK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {64, N, K / 128};
+  const cuuint64_t strides[2] = {K / 2, 64};
+  const cuuint32_t box[3] = {64, rows, (cuuint32_t)(K / 128)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(w), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CK_ERR_CUDA, "cuTensorMapEncodeTiled (weight tiles) failed (%d)", (int)r);
+  return CK_OK;
+}
+
+// Shared-memory layout of w4a8_stream_m8_kernel: as many 1024-aligned weight
+// stages as fit, then kRed partial-sum slots, the misc block and the barriers.
+ck::gstream::Layout stream_layout_m8(int stage_bytes, int misc_bytes);
+
 // Dynamic shared memory of one streaming-GEMV CTA: two CTAs (plus the 1 KB
 // the runtime reserves per CTA) fit in an SM's 228 KB.
 constexpr int kStreamSmemMax = 112 * 1024;
@@ -124,6 +146,20 @@ cudaError_t set_smem_max(KernelT kern, int bytes) {
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
   if (e == cudaSuccess) done[dev] = kStreamSmemMax;
   return e;
+}
+
+ck::gstream::Layout stream_layout_m8(int stage_bytes, int misc_bytes) {
+  using namespace ck::gstream;
+  Layout L;
+  L.stage_bytes = (stage_bytes + 1023) / 1024 * 1024;   // swizzled tile copies start on 1024-byte boundaries
+  const int bar_bytes = (2 * kMaxStages + 2 * kRed) * 8;
+  const int budget = kStreamSmemMax - 1024 - kRed * kRedBytes - misc_bytes - bar_bytes - 256;   // 1024: base alignment
+  L.ns = std::min(kMaxStages, budget / L.stage_bytes);
+  L.off_red = L.ns * L.stage_bytes;
+  L.off_misc = L.off_red + kRed * kRedBytes;
+  L.off_bar = (L.off_misc + misc_bytes + 15) / 16 * 16;
+  L.total = L.off_bar + bar_bytes + 1024;   // the kernel aligns its base up to 1024 bytes
+  return L;
 }
 
 // Shared-memory layout of a streaming GEMV: as many stages as fit in half of
@@ -614,6 +650,36 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
   const auto* sw = reinterpret_cast<const __nv_bfloat16*>(w_scale);
   const auto* bb = reinterpret_cast<const __nv_bfloat16*>(bias);
   auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
+  if (K <= 4096 && M <= 8) {
+    // streaming path for up to 8 activation rows: 16-row weight tiles as the m16 operand
+    using namespace ck::gstream;
+    W4A8Params sp;
+    sp.xq = xq; sp.xs = x_scale; sp.w = w_packed; sp.sw = sw; sp.bias = bb; sp.y = yy;
+    sp.M = (int)M; sp.K = (int)K; sp.N = (int)N;
+    sp.ntiles = (int)((N + 15) / 16);
+    const int grid = std::min(sp.ntiles, sm_count());
+    const int tpc = (sp.ntiles + grid - 1) / grid;
+    CUtensorMap tw;
+    ck_status r = make_tmap_wtile(&tw, w_packed, (uint64_t)N, (uint64_t)K, 16);
+    if (r != CK_OK) return r;
+    sp.L = stream_layout_m8((int)(16 * (K / 2)), kCons * 8 * 4 + 2 * 16 * tpc * 4 + 16);
+    const int nchunk = (int)(K / 128), cpw = (nchunk + kCons - 1) / kCons;
+    cudaError_t e;
+#define CK_W4A8_STREAM_M8(CPW)                                                                   \
+    {                                                                                            \
+      auto kern = w4a8_stream_m8_kernel<CPW>;                                                    \
+      struct Tag {};                                                                             \
+      e = set_smem_max<Tag>(kern, sp.L.total);                                                   \
+      if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), sp.L.total, S(stream), tw, sp); \
+    }
+    if (cpw <= 1) CK_W4A8_STREAM_M8(1)
+    else if (cpw == 2) CK_W4A8_STREAM_M8(2)
+    else if (cpw == 3) CK_W4A8_STREAM_M8(3)
+    else CK_W4A8_STREAM_M8(4)
+#undef CK_W4A8_STREAM_M8
+    if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
+    return launch_status("gemv_w4a8");
+  }
   if (K <= 4096) {
     // streaming path: 8-row weight tiles through a shared-memory ring, one CTA per SM
     using namespace ck::gstream;

@@ -14,6 +14,12 @@
 //              applies the scales and writes y.
 // All barrier waits are bounded; a timeout sets the device error word.
 //
+// For W4A8 with at most 8 activation rows, w4a8_stream_m8_kernel swaps the
+// MMA operands (16 weight rows as the m16 operand) and moves each 16-row tile
+// with ONE tensor copy through a 3-D view of the weight matrix (see
+// wtile_addr); it also hands a weight stage back as soon as it has been read,
+// with the partial sums passing through their own small ring.
+//
 // Back-to-back calls overlap: a CTA takes at most half of an SM's shared
 // memory, the kernels are launched as programmatic dependents, each lets the
 // next one be scheduled as soon as it starts, and a new call streams its first
@@ -47,6 +53,8 @@ constexpr int kCons = 8;
 constexpr int W_PROD = kCons, W_EPI = kCons + 1;
 constexpr int kThreads = (kCons + 2) * 32;
 constexpr int kMaxStages = 8;
+constexpr int kRed = 3;          // partial-sum slots of w4a8_stream_m8_kernel
+constexpr int kRedBytes = kCons * 32 * 4 * 4;
 
 // Shared-memory layout, computed on the host: [stages][red][misc][barriers].
 struct Layout {
@@ -57,6 +65,22 @@ struct Layout {
   int off_bar;
   int total;
 };
+
+// Tiles of w4a8_stream_m8_kernel: small copies are slow on this hardware (a
+// 2 KB bulk copy per weight row runs at a fraction of HBM bandwidth), so a
+// 16-row tile moves in one copy through a 3-D view of the weight matrix:
+// 64-byte slices of the rows outermost, the tile's rows in the middle. It
+// lands as [slice][row][64 B] with the 64-byte swizzle, which XORs each row's
+// 16-byte chunks with (row >> 1) & 3, so MMA-fragment reads of eight rows at
+// the same k hit different banks.
+// Shared-memory address of byte b of weight row r in a tile of R rows copied
+// as [b / 64][r][64 B] with the 64-byte swizzle (16-byte chunk c of a 64-byte
+// line L stored at chunk c ^ ((L >> 1) & 3); R even, so (L >> 1) & 3 only
+// depends on r).
+template <int R>
+__device__ __forceinline__ int wtile_addr(int r, int b) {
+  return ((b >> 6) * R + r) * 64 + ((((b >> 4) & 3) ^ ((r >> 1) & 3)) << 4) + (b & 15);
+}
 
 __device__ __forceinline__ void mma_s8u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -245,6 +269,200 @@ __global__ void __launch_bounds__(kThreads, 2) w4a8_stream_kernel(const W4A8Para
           const int a = acc[k] - 8 * ((k >> 1) ? xsg8 : xsg);
           float v = __fmul_rn(__fmul_rn((float)a, (k >> 1) ? sg8 : sg), colv[rl]);
           if (has_bias) v = __fadd_rn(v, colv[cb + rl]);
+          p.y[(int64_t)token * p.N + n] = __float2bfloat16_rn(v);
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// ============================================== W4A8, at most 8 activation rows
+
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The same product with the operands' roles swapped, for M <= 8: 16 weight
+// rows per tile are the m16 (unsigned) operand and the activation rows the n8
+// operand, so every MMA spends half of its work on real rows instead of
+// 1/16 .. 1/4 (the legacy mma.sync path has little throughput to spare).
+// Each lane holds, per 128-column chunk, the 16 bytes of weight rows g and
+// g + 8 at k = 32t .. 32t + 31 of the chunk; MMA step j takes word j of them,
+// its low nibbles (even k) in fragment slots 4t..4t+3 and its high nibbles
+// (odd k) in slots 16+4t..16+4t+3; the activation fragments follow the same
+// k order. Shared memory: [ns weight stages][kRed partial-sum slots][misc]
+// [barriers full, wfree (kMaxStages); rfull, rfree (kRed)]: a weight stage is
+// refilled once every consumer warp has read it; the epilogue reduces the
+// partial sums from their own ring.
+template <int CPW>   // 128-column chunks per consumer warp (K <= 8 * 128 * CPW)
+__global__ void __launch_bounds__(kThreads, 2)
+    w4a8_stream_m8_kernel(const __grid_constant__ CUtensorMap tm_w, const W4A8Params p) {
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  const Layout& L = p.L;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.off_bar);
+  uint64_t* wfree = full + kMaxStages;
+  uint64_t* rfull = wfree + kMaxStages;
+  uint64_t* rfree = rfull + kRed;
+  int* red = reinterpret_cast<int*>(sm + L.off_red);
+  int* xsum_part = reinterpret_cast<int*>(sm + L.off_misc);           // [kCons][8]
+  float* colv = reinterpret_cast<float*>(xsum_part + kCons * 8);      // [2][rows of this CTA]
+  const int rows_cta = 16 * ((p.ntiles + gridDim.x - 1) / gridDim.x);
+  int* abort_flag = reinterpret_cast<int*>(colv + 2 * rows_cta);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int t0 = (int)((int64_t)blockIdx.x * p.ntiles / gridDim.x);
+  const int t1 = (int)((int64_t)(blockIdx.x + 1) * p.ntiles / gridDim.x);
+  const int nt = t1 - t0;
+  const int wld = p.K >> 1;
+  const int nchunk = p.K >> 7;
+  const int ns = L.ns;
+
+  auto issue = [&](int i) {   // rows past N arrive as zeros (and are never stored)
+    const int s = i % ns;
+    mbar_arrive_expect_tx(&full[s], (uint32_t)(16 * wld));
+    tma_load_3d(sm + s * L.stage_bytes, &tm_w, &full[s], 0, 16 * (t0 + i), 0);
+  };
+  if (warp == W_PROD && lane == 0) {
+    prefetch_tmap(&tm_w);
+    for (int s = 0; s < ns; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&wfree[s], kCons);
+    }
+    for (int r = 0; r < kRed; ++r) {
+      mbar_init(&rfull[r], kCons);
+      mbar_init(&rfree[r], 1);
+    }
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    for (int i = 0; i < min(ns, nt); ++i) issue(i);
+  }
+  grid_dep_launch();
+  grid_dep_wait();   // the activations and the output belong to the previous kernel until here
+
+  uint32_t bf[CPW][4][2];   // activation fragments of token g
+  if (warp < kCons) {
+    int xs_g = 0;
+#pragma unroll
+    for (int ci = 0; ci < CPW; ++ci) {
+      const int c = warp + kCons * ci;
+      uint4 a0 = make_uint4(0, 0, 0, 0), a1 = a0;
+      if (c < nchunk && g < p.M) {
+        const uint4* xp = reinterpret_cast<const uint4*>(p.xq + (int64_t)g * p.K + c * 128 + 32 * t);
+        a0 = __ldg(xp);
+        a1 = __ldg(xp + 1);
+      }
+      const uint32_t xa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) xs_g = __dp4a((int)xa[q], 0x01010101, xs_g);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {   // k = c*128 + 32t + 8j + (0 2 4 6) and + (1 3 5 7)
+        bf[ci][j][0] = __byte_perm(xa[2 * j], xa[2 * j + 1], 0x6420);
+        bf[ci][j][1] = __byte_perm(xa[2 * j], xa[2 * j + 1], 0x7531);
+      }
+    }
+    xs_g += __shfl_xor_sync(0xffffffffu, xs_g, 1);
+    xs_g += __shfl_xor_sync(0xffffffffu, xs_g, 2);
+    if (t == 0) xsum_part[warp * 8 + g] = xs_g;
+  } else if (warp == W_EPI) {
+    const int r0 = 16 * t0, nr = min(16 * nt, p.N - r0);
+    for (int r = lane; r < nr; r += 32) {
+      colv[r] = __bfloat162float(p.sw[r0 + r]);
+      colv[rows_cta + r] = p.bias ? __bfloat162float(p.bias[r0 + r]) : 0.0f;
+    }
+  }
+  __syncthreads();
+  volatile int* abort = abort_flag;
+
+  if (warp < kCons) {
+    // = wtile_addr<16>(g, c * 64 + 16 * t) for c = warp + 8 * ci; row g + 8 is 8 lines on
+    const int wb = (warp * 16 + g) * 64 + ((t ^ ((g >> 1) & 3)) << 4);
+    for (int i = 0; i < nt; ++i) {
+      const int s = i % ns, rs = i % kRed;
+      if (!warp_wait(&full[s], (i / ns) & 1, abort, 30)) break;
+      const uint8_t* st = sm + s * L.stage_bytes;
+      uint4 wg[CPW], wg8[CPW];
+#pragma unroll
+      for (int ci = 0; ci < CPW; ++ci) {
+        const bool live = warp + kCons * ci < nchunk;
+        wg[ci] = live ? *reinterpret_cast<const uint4*>(st + wb + 8192 * ci) : make_uint4(0, 0, 0, 0);
+        wg8[ci] = live ? *reinterpret_cast<const uint4*>(st + wb + 8192 * ci + 512) : make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wfree[s]);
+      int accc[CPW][4];
+#pragma unroll
+      for (int ci = 0; ci < CPW; ++ci) {
+        accc[ci][0] = accc[ci][1] = accc[ci][2] = accc[ci][3] = 0;
+        if (warp + kCons * ci < nchunk) {
+          const uint32_t u[4] = {wg[ci].x, wg[ci].y, wg[ci].z, wg[ci].w};
+          const uint32_t v[4] = {wg8[ci].x, wg8[ci].y, wg8[ci].z, wg8[ci].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t a[4] = {u[j] & 0x0F0F0F0Fu, v[j] & 0x0F0F0F0Fu, (u[j] >> 4) & 0x0F0F0F0Fu,
+                                   (v[j] >> 4) & 0x0F0F0F0Fu};
+            mma_u8s8(accc[ci], a, bf[ci][j][0], bf[ci][j][1]);
+          }
+        }
+      }
+      int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int ci = 0; ci < CPW; ++ci) {
+        acc[0] += accc[ci][0]; acc[1] += accc[ci][1]; acc[2] += accc[ci][2]; acc[3] += accc[ci][3];
+      }
+      if (!warp_wait(&rfree[rs], ((i / kRed) & 1) ^ 1, abort, 31)) break;
+      *reinterpret_cast<int4*>(red + ((rs * kCons + warp) * 32 + lane) * 4) = make_int4(acc[0], acc[1], acc[2], acc[3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfull[rs]);
+    }
+  } else if (warp == W_PROD) {
+    if (lane == 0) {
+      int issued = min(ns, nt);
+      for (int i = issued; i < nt; ++i) {
+        if (!mbar_wait(&wfree[i % ns], ((i / ns) & 1) ^ 1, abort, 32)) break;
+        issue(i);
+        issued = i + 1;
+      }
+      if (*abort)
+        for (int i = issued - 1; i >= 0 && i >= issued - ns; --i)
+          mbar_wait(&full[i % ns], (i / ns) & 1, nullptr, 33, 100000000ull);
+    }
+  } else {
+    // epilogue: lane (g, t) finishes weight rows g, g + 8 x tokens 2t, 2t + 1 of each tile
+    int xs2[2] = {0, 0};
+#pragma unroll
+    for (int w = 0; w < kCons; ++w) {
+      xs2[0] += xsum_part[w * 8 + 2 * t];
+      xs2[1] += xsum_part[w * 8 + 2 * t + 1];
+    }
+    const float sx[2] = {2 * t < p.M ? p.xs[2 * t] : 0.0f, 2 * t + 1 < p.M ? p.xs[2 * t + 1] : 0.0f};
+    const bool has_bias = p.bias != nullptr;
+    for (int i = 0; i < nt; ++i) {
+      const int rs = i % kRed;
+      if (!warp_wait(&rfull[rs], (i / kRed) & 1, abort, 34)) break;
+      int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int w = 0; w < kCons; ++w) {
+        const int4 v = *reinterpret_cast<const int4*>(red + ((rs * kCons + w) * 32 + lane) * 4);
+        acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfree[rs]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int token = 2 * t + (k & 1);
+        const int rl = 16 * i + g + 8 * (k >> 1);           // row within this CTA's range
+        const int n = 16 * t0 + rl;
+        if (token < p.M && n < p.N) {
+          const int a = acc[k] - 8 * xs2[k & 1];
+          float v = __fmul_rn(__fmul_rn((float)a, sx[k & 1]), colv[rl]);
+          if (has_bias) v = __fadd_rn(v, colv[rows_cta + rl]);
           p.y[(int64_t)token * p.N + n] = __float2bfloat16_rn(v);
         }
       }
