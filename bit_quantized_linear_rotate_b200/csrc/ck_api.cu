@@ -730,7 +730,8 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
   if (!aligned(x, 16) || !aligned(qweight, 16)) return fail(CK_ERR_UNSUPPORTED, "gemv_awq_w4a16: x and qweight must be 16-byte aligned");
   if (!aligned(wscales, 2) || !aligned(wzeros, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "gemv_awq_w4a16: misaligned scales, zeros, bias or output");
-  if (K <= 4096 && K / group_size <= 256 && N % 8 == 0 && aligned(wscales, 16) && aligned(wzeros, 16)) {
+  if (K <= 4096 && K / group_size <= 256 && N % 8 == 0 && is_pow2(group_size / 64) && aligned(wscales, 16) &&
+      aligned(wzeros, 16)) {
     // streaming path: 16-row weight tiles plus their scales and zeros through a shared-memory ring
     using namespace ck::gstream;
     CUtensorMap ts, tz;
@@ -744,6 +745,8 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
     AwqParams ap;
     ap.x = x; ap.qw = qweight; ap.bias = bias; ap.y = y;
     ap.M = (int)M; ap.K = (int)K; ap.N = (int)N; ap.G = group_size;
+    ap.gshift = 0;
+    while ((64 << ap.gshift) < group_size) ++ap.gshift;
     ap.ntiles = (int)((N + 15) / 16);
     ap.srow = (int)(K / 2) + 32;
     ap.w_bytes = (16 * ap.srow + 127) / 128 * 128;    // padded rows; the scale tiles follow 128-byte aligned

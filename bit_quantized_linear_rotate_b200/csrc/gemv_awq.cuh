@@ -74,6 +74,18 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int s) {
   return Traits<T>::sub2(((w >> (4 * s)) & 0x000F000Fu) | Traits<T>::kMagic, Traits<T>::kBias);
 }
 
+// The same pair without the subtraction: (128 + u) as bf16, (1024 + u) as
+// fp16, one shift and one logical op. A sum of such products carries an
+// extra kOffset * sum(x), which the streaming kernel removes with the group's
+// zero term: s * (P' - kOffset X) + z X = s P' + (z - kOffset s) X.
+template <typename T>
+__device__ __forceinline__ uint32_t nib_pair_raw(uint32_t w, int s) {
+  return ((w >> (4 * s)) & 0x000F000Fu) | Traits<T>::kMagic;
+}
+template <typename T> struct RawOffset;
+template <> struct RawOffset<__nv_bfloat16> { static constexpr float v = 136.0f; };   // 128 + 8
+template <> struct RawOffset<__half> { static constexpr float v = 1032.0f; };         // 1024 + 8
+
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32) gemv_awq_kernel(
     const T* __restrict__ x, int M, int K, int N, int G, const uint8_t* __restrict__ qw,

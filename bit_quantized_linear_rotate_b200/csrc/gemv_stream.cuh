@@ -479,6 +479,7 @@ struct AwqParams {
   const void* bias;              // (N) T or null
   void* y;                       // (M, N) T
   int M, K, N, G;
+  int gshift;                    // log2(G / 64): 64-column sub-block -> quantization group
   int ntiles;                    // 16-row weight tiles
   int w_bytes;                   // 16 * K / 2
   int sz_bytes;                  // (K / G) * 16 * 2: one of scales / zeros per stage
@@ -587,20 +588,23 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint2 w0 = *reinterpret_cast<const uint2*>(st + g * p.srow + sb * 32 + 8 * t);
           const uint2 w1 = *reinterpret_cast<const uint2*>(st + (g + 8) * p.srow + sb * 32 + 8 * t);
           const uint32_t r0[2] = {w0.x, w0.y}, r1[2] = {w1.x, w1.y};
+          // weights enter the MMA as (offset + u); the group's zero term takes the offset back out
           float P[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int wd = j >> 1, s0 = (2 * j) & 3, s1 = (2 * j + 1) & 3;
             uint32_t a[4];
-            a[0] = awq::nib_pair<T>(r0[wd], s0);
-            a[1] = awq::nib_pair<T>(r1[wd], s0);
-            a[2] = awq::nib_pair<T>(r0[wd], s1);
-            a[3] = awq::nib_pair<T>(r1[wd], s1);
+            a[0] = awq::nib_pair_raw<T>(r0[wd], s0);
+            a[1] = awq::nib_pair_raw<T>(r1[wd], s0);
+            a[2] = awq::nib_pair_raw<T>(r0[wd], s1);
+            a[3] = awq::nib_pair_raw<T>(r1[wd], s1);
             Tr::mma(P, a, bp[i2][2 * j], bp[i2][2 * j + 1]);
           }
-          const int grp = (sb * 64) / p.G;
-          const float sa = Tr::tof(sc[grp * 16 + g]), za = Tr::tof(zr[grp * 16 + g]);
-          const float sbb = Tr::tof(sc[grp * 16 + g + 8]), zb = Tr::tof(zr[grp * 16 + g + 8]);
+          const int grp = sb >> p.gshift;
+          constexpr float kOff = awq::RawOffset<T>::v;
+          const float sa = Tr::tof(sc[grp * 16 + g]), sbb = Tr::tof(sc[grp * 16 + g + 8]);
+          const float za = fmaf(-kOff, sa, Tr::tof(zr[grp * 16 + g]));
+          const float zb = fmaf(-kOff, sbb, Tr::tof(zr[grp * 16 + g + 8]));
           yacc[0] += sa * P[0] + za * X[i2][0];
           yacc[1] += sa * P[1] + za * X[i2][1];
           yacc[2] += sbb * P[2] + zb * X[i2][0];
