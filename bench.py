@@ -348,7 +348,7 @@ def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
         out[f"w4a8_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
                              "all_GBps": allb / (ms * 1e-3) / 1e9,
                              "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R,
-                             "traffic": load_traffic("w4a8_stream_kernel") if M == 16 else None}
+                             "traffic": load_traffic("w4a8_stream_m8_kernel" if M <= 8 else "w4a8_stream_kernel")}
     w = WL.GEMV_AWQ
     for M in w.Ms:
         d = WL.gemv_awq_inputs(w, M)
@@ -366,7 +366,7 @@ def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
         out[f"awq_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
                             "all_GBps": allb / (ms * 1e-3) / 1e9,
                             "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R,
-                            "traffic": load_traffic("awq_stream_kernel") if M == 4 else None}
+                            "traffic": load_traffic("awq_stream_kernel")}
     return out
 
 
