@@ -37,6 +37,7 @@ _int = ctypes.c_int
 SIGNATURES = {
     "ck_rotate_quant_rowwise": [_p, _int, _i64, _i64, _i64, _int, _int, _p, _p, _p],
     "ck_rotate_quant_rowwise_i8": [_p, _int, _i64, _i64, _i64, _int, _int, _p, _p, _p],
+    "ck_rotate_quant_rowwise_r": [_p, _int, _i64, _i64, _i64, _int, _p, _int, _p, _p, _p],
     "ck_gemm_w4a4": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemm_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_unpack_int4": [_p, _i64, _i64, _p, _p],
@@ -150,6 +151,28 @@ def rotate_quant_rowwise_i8(x, group_size: int, bits: int, q_out=None, scale_out
     _check(lib.ck_rotate_quant_rowwise_i8(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
                                           _ptr(q_out), _ptr(scale_out), _stream(stream)),
            "ck_rotate_quant_rowwise_i8")
+    return q_out, scale_out
+
+
+def rotate_quant_rowwise_r(x, R, bits: int, q_out=None, scale_out=None, stream=None):
+    """Rotation by a general (G, G) float32 matrix R (y_g = x_g @ R), then rowwise quantization.
+
+    Returns (q, s) in the formats of rotate_quant_rowwise: bits=4 packed (..., K/2) uint8, bits=8
+    (..., K) int8; s (...) float32.
+    """
+    _cuda(x, R)
+    if R.dtype != torch.float32 or R.dim() != 2 or R.shape[0] != R.shape[1] or not R.is_contiguous():
+        raise ValueError("R must be a contiguous square float32 matrix")
+    M, K, ldx, x2 = _rows(x)
+    lead = tuple(x.shape[:-1])
+    if q_out is None:
+        q_out = torch.empty(lead + ((K // 2,) if bits == 4 else (K,)), device=x.device,
+                            dtype=torch.uint8 if bits == 4 else torch.int8)
+    if scale_out is None:
+        scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
+    _check(lib.ck_rotate_quant_rowwise_r(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, R.shape[0], _ptr(R), bits,
+                                         _ptr(q_out), _ptr(scale_out), _stream(stream)),
+           "ck_rotate_quant_rowwise_r")
     return q_out, scale_out
 
 

@@ -21,6 +21,7 @@
 #include "gemv_stream.cuh"
 #include "gemv_w4a8.cuh"
 #include "rotate_quant.cuh"
+#include "rotate_quant_general.cuh"
 
 namespace {
 
@@ -442,6 +443,43 @@ ck_status ck_rotate_quant_rowwise_i8(const void* x, ck_dtype xt, int64_t M, int6
   if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "rotate_quant_i8: M too large");
   return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, ck::rq::STORE_INT8, q_out, scale_out, nullptr,
                            S(stream));
+}
+
+ck_status ck_rotate_quant_rowwise_r(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                    int group_size, const float* R, int bits, void* q_out, float* scale_out,
+                                    void* stream) {
+  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: unknown dtype");
+  if (bits != 4 && bits != 8) return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: bits must be 4 or 8");
+  if (M < 0 || K <= 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: M >= 0 and K > 0 required");
+  if (group_size < 1 || group_size > 256)
+    return fail(CK_ERR_UNSUPPORTED, "rotate_quant_rowwise_r: group_size=%d outside [1, 256]", group_size);
+  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: K %% group_size != 0");
+  if (K % 2 != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: K must be even");
+  if (K > 16384) return fail(CK_ERR_UNSUPPORTED, "rotate_quant_rowwise_r: K=%lld > 16384", (long long)K);
+  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: ldx < K");
+  if (M == 0) return ok();
+  if (!x || !R || !q_out || !scale_out) return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: null pointer");
+  if (!aligned(x, 2) || !aligned(R, 4) || !aligned(scale_out, 4))
+    return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: misaligned pointer");
+  const size_t smem = 2 * (size_t)K * sizeof(float);
+  const unsigned grid = (unsigned)std::min<int64_t>(M, 8 * (int64_t)sm_count());
+  cudaError_t e = cudaSuccess;
+#define CK_RQG(T, B)                                                                                 \
+  {                                                                                                  \
+    auto kern = ck::rqg::rotate_quant_general_kernel<T, B>;                                          \
+    if (smem > 48 * 1024) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (e == cudaSuccess)                                                                            \
+      e = launch_pdl(kern, dim3(grid), dim3(ck::rqg::kThreads), smem, S(stream), reinterpret_cast<const T*>(x), M, \
+                     (int)K, ldx, group_size, R, reinterpret_cast<uint8_t*>(q_out), scale_out);       \
+  }
+  if (xt == CK_BF16) {
+    if (bits == 4) CK_RQG(__nv_bfloat16, 4) else CK_RQG(__nv_bfloat16, 8)
+  } else {
+    if (bits == 4) CK_RQG(__half, 4) else CK_RQG(__half, 8)
+  }
+#undef CK_RQG
+  if (e != cudaSuccess) return fail(CK_ERR_CUDA, "rotate_quant_rowwise_r: %s", cudaGetErrorString(e));
+  return launch_status("rotate_quant_rowwise_r");
 }
 
 ck_status ck_unpack_int4(const uint8_t* packed, int64_t R, int64_t C, int8_t* out, void* stream) {

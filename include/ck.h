@@ -81,6 +81,22 @@ ck_status ck_rotate_quant_rowwise_i8(const void* x, ck_dtype xt, int64_t M, int6
                                      float* scale_out, void* stream);
 
 /*
+ * ck_rotate_quant_rowwise with a GENERAL rotation: y_g = x_g . R for every
+ * group g of every row, R any G x G matrix (the pages test
+ * quantize_and_rotate_rowwise with "asymmetric-rotation inputs", comfy-kitchen
+ * PR #155, "How was this patch tested?"), followed by the same rowwise
+ * symmetric quantization and the same output formats as
+ * ck_rotate_quant_rowwise. The product runs in fp32 on the CUDA cores (G
+ * multiply-adds per element): a functional path, not the Hadamard fast path.
+ * R          : (G, G) float32, row-major, device memory: y[j] = sum_i x[i] R[i][j].
+ * group_size : 1 .. 256 with K % group_size == 0; K even, K <= 16384.
+ * Other arguments as for ck_rotate_quant_rowwise (x 2-byte aligned suffices).
+ */
+ck_status ck_rotate_quant_rowwise_r(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                    int group_size, const float* R, int bits, void* q_out,
+                                    float* scale_out, void* stream);
+
+/*
  * Integer matmul of packed int4 activations with packed int4 weights, int32
  * accumulation on the tcgen05 tensor cores, and the rowwise-scale epilogue
  * (the "EpiRowwise" of comfy-kitchen PR #182, Description):

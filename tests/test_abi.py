@@ -126,6 +126,23 @@ def test_gemv_validation(ck):
     assert L.ck_gemv_awq_w4a16(P(1 << 20), 5, 2, 128, 8, 64, P(1 << 20), P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
 
 
+def test_general_rotation_validation(ck):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    ok = dict(x=P(1 << 20), xt=0, M=4, K=64, ldx=64, G=16, R=P(1 << 22), bits=4, q=P(1 << 21), s=P(1 << 23))
+    def call(**kw):
+        a = dict(ok); a.update(kw)
+        return L.ck_rotate_quant_rowwise_r(a["x"], a["xt"], a["M"], a["K"], a["ldx"], a["G"], a["R"], a["bits"],
+                                           a["q"], a["s"], None)
+    assert call(G=0) == ck.CK_ERR_UNSUPPORTED
+    assert call(G=512, K=512, ldx=512) == ck.CK_ERR_UNSUPPORTED
+    assert call(G=48) == ck.CK_ERR_INVALID_ARG          # K % G != 0
+    assert call(bits=2) == ck.CK_ERR_INVALID_ARG
+    assert call(R=None) == ck.CK_ERR_INVALID_ARG
+    assert call(K=63, ldx=64, G=1) == ck.CK_ERR_INVALID_ARG   # K odd
+    assert call(M=0, x=None, R=None, q=None, s=None) == ck.CK_OK
+
+
 def test_selftest_timeout_range_is_validated(ck):
     assert ck.lib.ck_selftest_bounded_wait(10, None) == ck.CK_ERR_INVALID_ARG
     assert ck.lib.ck_selftest_bounded_wait(10 ** 10, None) == ck.CK_ERR_INVALID_ARG

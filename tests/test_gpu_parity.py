@@ -59,6 +59,36 @@ def test_rotate_quant_matches_oracle(ck, G, bits, dtype):
         assert np.array_equal(same[agree], np.ones(int(agree.sum()), dtype=bool))
 
 
+@pytest.mark.parametrize("G,bits,dtype", [(16, 4, torch.bfloat16), (64, 8, torch.float16), (256, 4, torch.bfloat16),
+                                          (3, 8, torch.bfloat16), (1, 4, torch.float16)])
+def test_rotate_quant_general_R_matches_oracle(ck, G, bits, dtype):
+    # a general rotation: non-symmetric, not orthogonal (y_g = x_g @ R)
+    M, K = 37, 768 if G != 3 else 768 - 768 % 6
+    xf = _rand_x(M, K + 32, seed=G * 7 + bits, dtype=dtype, outliers=4)
+    xf[5] = 0                                    # an all-zero row gets scale 1
+    g = torch.Generator().manual_seed(G)
+    R = (torch.randn(G, G, generator=g, dtype=torch.float64) / max(G, 1) ** 0.5).float()
+    x = xf.to(DEV)[:, :K]
+    q, s = ck.rotate_quant_rowwise_r(x, R.to(DEV), bits)
+    torch.cuda.synchronize()
+    q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf[:, :K]), G, bits, R.double().numpy())
+    assert s[5].item() == 1.0
+    assert_scales_close(s.cpu().numpy(), s_ref)
+    assert_codes_close(unpack_codes(q) if bits == 4 else q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("G", [16, 64, 256])
+def test_rotate_quant_general_R_with_hadamard_equals_fast_path(ck, G):
+    M, K = 64, 1024
+    x = _rand_x(M, K, seed=G, outliers=4).to(DEV)
+    H = torch.tensor(O.hadamard_sylvester(G), dtype=torch.float32, device=DEV)
+    qg, sg = ck.rotate_quant_rowwise_r(x, H, 8)
+    qf, sf = ck.rotate_quant_rowwise(x, G, 8)
+    torch.cuda.synchronize()
+    assert_scales_close(sg.cpu().numpy(), sf.cpu().numpy().astype(np.float32))
+    assert_codes_close(qg.cpu().numpy(), qf.cpu().numpy())
+
+
 @pytest.mark.parametrize("G", [1, 2, 8, 32, 128])
 def test_rotate_quant_other_group_sizes(ck, G):
     M, K = 19, 1024
@@ -429,3 +459,68 @@ def test_invalid_arguments_raise(ck):
         ck.gemv_w4a8(torch.zeros(17, 128, device=DEV, dtype=torch.int8), torch.ones(17, device=DEV),
                      torch.zeros(8, 64, device=DEV, dtype=torch.uint8), torch.ones(8, device=DEV, dtype=torch.bfloat16))
     assert e.value.status == ck.CK_ERR_UNSUPPORTED
+
+
+# ------------------------------------ back-to-back calls (programmatic dependents)
+
+def test_back_to_back_linear_calls_share_a_workspace(ck):
+    """Consecutive linears on one stream reuse one workspace with no host sync in between: the
+    next call's rotate+quant may only overwrite the workspace once the previous GEMM is done."""
+    M, K, N, G = 1024, 3840, 3840, 64
+    ins = [WL.small_linear_inputs(M, K, N, 40 + i, n_outlier_cols=8) for i in range(4)]
+    ds = [{k: v.to(DEV) for k, v in d.items()} for d in ins]
+    refs = []
+    for d in ds:   # one call at a time, synchronised
+        refs.append(ck.linear_w4a4(d["x"], d["w_packed"], d["w_scale"], G).clone())
+        torch.cuda.synchronize()
+    ws = torch.empty(ck.linear_w4a4_workspace_bytes(M, K), device=DEV, dtype=torch.uint8)
+    outs = [torch.empty(M, N, device=DEV, dtype=torch.bfloat16) for _ in ds]
+    for rep in range(3):
+        for d, o in zip(ds, outs):
+            ck.linear_w4a4(d["x"], d["w_packed"], d["w_scale"], G, workspace=ws, out=o)
+    torch.cuda.synchronize()
+    for o, r in zip(outs, refs):
+        assert torch.equal(o.view(torch.int16), r.view(torch.int16))
+    ck.device_error_check()
+
+
+def test_back_to_back_dependent_gemvs(ck):
+    """A chain of GEMVs where each call reads the previous call's output, launched back to back:
+    every activation read must see the previous kernel's writes."""
+    K = N = 1024
+    g = torch.Generator().manual_seed(77)
+    x0 = WL.activations(2, K, 0, g)
+    layers = []
+    for _ in range(4):
+        qw = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+        ws_ = WL.uniform((K // 64, N), 0.001, 0.01, g)
+        wz = (torch.randn((K // 64, N), generator=g) * 0.01).to(torch.bfloat16)
+        layers.append((qw.to(DEV), ws_.to(DEV), wz.to(DEV)))
+    # chained without syncs
+    y = x0.to(DEV)
+    for qw, ws_, wz in layers:
+        y = ck.gemv_awq_w4a16(y, qw, ws_, wz, group_size=64)
+    torch.cuda.synchronize()
+    chained = y.clone()
+    # the same chain with a sync after every call
+    y = x0.to(DEV)
+    for qw, ws_, wz in layers:
+        y = ck.gemv_awq_w4a16(y, qw, ws_, wz, group_size=64)
+        torch.cuda.synchronize()
+    assert torch.equal(chained.view(torch.int16), y.view(torch.int16))
+    # and the W4A8 GEMV reading codes that rotate_quant_rowwise (G = 1, int8) writes just before
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8).to(DEV)
+    sw = WL.uniform((N,), 0.005, 0.02, g).to(DEV)
+    xs = [WL.activations(4, K, 0, g).to(DEV) for _ in range(3)]
+    outs = []
+    for xx in xs:
+        xq, xsc = ck.rotate_quant_rowwise(xx, 1, 8)
+        outs.append(ck.gemv_w4a8(xq, xsc, wp, sw))
+    torch.cuda.synchronize()
+    for xx, o in zip(xs, outs):
+        xq, xsc = ck.rotate_quant_rowwise(xx, 1, 8)
+        torch.cuda.synchronize()
+        r = ck.gemv_w4a8(xq, xsc, wp, sw)
+        torch.cuda.synchronize()
+        assert torch.equal(o.view(torch.int16), r.view(torch.int16))
+    ck.device_error_check()
