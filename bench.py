@@ -55,24 +55,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
+    """Hash of the named files under csrc/ (a kernel's own header and the device helpers it uses)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "bit_quantized_linear_rotate_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def load_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if taken on this exact source."""
+    """DRAM bytes per launch from the committed ncu summary, if taken on this kernel's exact sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("sources", [])):
         return None
     return e.get("dram_bytes_per_launch")
 
