@@ -394,6 +394,48 @@ def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
     return out
 
 
+def time_other_configs(ck, dev, peaks):
+    """The other linear workloads and the standalone rotate+quant at the pages' shapes.
+
+    Graph-replayed over rotating input copies (no copy stays in L2 between calls)."""
+    out = {}
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    for w in (WL.LINEAR_M32, WL.LINEAR_MLP_DOWN):
+        d = WL.linear_inputs(w)
+        per = d["x"].numel() * 2 + d["w_packed"].numel()
+        R = max(2, -(-2 * L2_BYTES // per))
+        xs = [d["x"].to(dev) for _ in range(R)]
+        wps = [d["w_packed"].to(dev) for _ in range(R)]
+        sw = d["w_scale"].to(dev)
+        y = torch.empty(w.M, w.N, device=dev, dtype=torch.bfloat16)
+        ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
+        ms = time_rotating(lambda c: ck.linear_w4a4(xs[c], wps[c], sw, w.G, workspace=ws, out=y), R, 100, 5)
+        ops = 2.0 * w.M * w.N * w.K
+        out[w.name] = {"us": round(ms * 1e3, 2), "TOPS": round(ops / (ms * 1e-3) / 1e12, 1),
+                       "frac_int8": round(ops / (ms * 1e-3) / 1e12 / int8_peak, 4),
+                       "weight_GBps": round(d["w_packed"].numel() / (ms * 1e-3) / 1e9, 1), "copies": R}
+        del xs, wps
+    # rotate+quant (int8 codes, as the pages' RotateQuant measures) at the pages' activation shapes,
+    # plus the MLP-down standalone case (G = 16, bits 4 and 8)
+    cases = [(32, 3840, 64, 8), (8192, 3840, 64, 8), (32, 10240, 64, 8), (8192, 10240, 64, 8),
+             (8192, 10240, 16, 8), (8192, 10240, 16, 4)]
+    for M, K, G, bits in cases:
+        g = torch.Generator().manual_seed(M + K + G)
+        x0 = WL.activations(M, K, max(1, K // 100), g)
+        R = max(2, -(-2 * L2_BYTES // (x0.numel() * 2)))
+        xs = [x0.to(dev) for _ in range(R)]
+        q = torch.empty((M, K // 2) if bits == 4 else (M, K), device=dev,
+                        dtype=torch.uint8 if bits == 4 else torch.int8)
+        sc = torch.empty(M, device=dev, dtype=torch.float32)
+        ms = time_rotating(lambda c: ck.rotate_quant_rowwise(xs[c], G, bits, q_out=q, scale_out=sc), R, 100, 5)
+        nbytes = M * K * 2 + q.numel() + 4 * M
+        out[f"rotate_quant_M{M}_K{K}_G{G}_int{bits}"] = {
+            "us": round(ms * 1e3, 2), "GBps": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "copies": R}
+        del xs
+    return out
+
+
 # --------------------------------------------------------------------- arms
 
 def run_ours(args, world, rank, local):
@@ -436,6 +478,7 @@ def run_ours(args, world, rank, local):
         line["e2e"] = time_linear_e2e(ck, w, max(3, min(args.steps, 50)), 3, dev)
     if not args.skip_siblings:
         line["siblings"] = time_gemvs(ck, dev, peaks["hbm_gbs"])
+        line["other_configs"] = time_other_configs(ck, dev, peaks)
     if rank == 0 and world == 1 and not args.skip_cpu:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
     if rank == 0:

@@ -387,6 +387,16 @@ size_t linear_ws_bytes(int64_t M, int64_t K) {
   return linear_q_bytes(M, K) + align256((size_t)M * sizeof(float)) + (size_t)M * sizeof(int32_t);
 }
 
+// Small batches of the linear take the decode-GEMV kernels instead of the
+// tensor-core GEMM: with M <= 64 the GEMM's 256 x 256 pair tiles leave most
+// SMs idle (K = N = 3840: 15 of 74 pairs busy), while the streaming GEMV
+// spreads the weights over every SM. The codes then stay in natural column
+// order (the GEMV computes its own row sums). The epilogue arithmetic is the
+// same, so the results do not depend on the route. Both phases of the linear
+// take the decision from (M, K) alone.
+bool linear_small_m(int64_t M, int64_t K) { return M <= 64 && K % 128 == 0 && K <= 4096; }
+constexpr int64_t kSmallMChunk = 16;   // rows per GEMV call
+
 ck_status check_linear_workspace(const char* who, int64_t M, int64_t K, const void* ws, size_t bytes) {
   if (ws == nullptr || bytes < linear_ws_bytes(M, K))
     return fail(CK_ERR_INVALID_ARG, "%s: workspace smaller than ck_linear_w4a4_workspace_bytes", who);
@@ -559,8 +569,8 @@ ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t
   if (x == nullptr) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: null pointer");
   if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: x rows must be 16-byte aligned");
   LinearWs ws = linear_ws(workspace, M, K);
-  return rotate_quant_impl(x, xt, M, K, ldx, group_size, 4, ck::rq::STORE_INT8_PERM, ws.q, ws.scale, ws.rowsum,
-                           S(stream));
+  const int store = linear_small_m(M, K) ? ck::rq::STORE_INT8 : ck::rq::STORE_INT8_PERM;
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, 4, store, ws.q, ws.scale, ws.rowsum, S(stream));
 }
 
 ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
@@ -574,6 +584,14 @@ ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* 
   if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "linear_w4a4_matmul: misaligned scale, bias or output");
   LinearWs ws = linear_ws(const_cast<void*>(workspace), M, K);
+  if (linear_small_m(M, K)) {
+    for (int64_t r0 = 0; r0 < M; r0 += kSmallMChunk) {
+      const int64_t mc = std::min<int64_t>(kSmallMChunk, M - r0);
+      r = ck_gemv_w4a8(ws.q + r0 * K, ws.scale + r0, mc, K, N, w_packed, w_scale, bias, y + r0 * N, stream);
+      if (r != CK_OK) return r;
+    }
+    return ok();
+  }
   return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4_U, ck::gemm::EPI_BF16>(
       ws.q, M, K, N, w_packed, ws.scale, ws.rowsum, w_scale, bias, y, S(stream));
 }
