@@ -170,12 +170,15 @@ ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64
 
 /*
  * The two phases of ck_linear_w4a4, callable separately (to time or overlap
- * them). Phase 1 rotates and quantizes x into `workspace` (the int4 codes
- * stored one per byte, as comfy-kitchen PR #212 "Related work" notes #201
- * does away with the activation pack/unpack, in the column order the GEMM's
- * weight decode produces, with the row scales and the row sums of the codes).
- * Phase 2 runs the tensor-core GEMM of those codes against the packed int4
- * weights and the rowwise-scale epilogue.
+ * them). Phase 1 rotates and quantizes x into `workspace`: the int4 codes
+ * stored one per byte (as comfy-kitchen PR #212 "Related work" notes, #201
+ * does away with the activation pack/unpack) and the row scales, in a layout
+ * private to the library that depends only on (M, K). Phase 2 multiplies
+ * those codes with the packed int4 weights and applies the rowwise-scale
+ * epilogue: on the tensor-core GEMM, or for small batches (M <= 64, K <= 4096,
+ * K % 128 == 0) on the streaming decode-GEMV kernels, which keep every SM
+ * busy at such M. The result does not depend on the route. Call both phases
+ * with the same M and K.
  */
 ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
                                   int group_size, void* workspace, size_t ws_bytes, void* stream);
