@@ -34,6 +34,11 @@ Readings where the pages are silent (each is repeated in the design doc):
 * Rounding: round half to even of y / s (float64 division), then clamp.
 * Codec: offset binary, nibble u = q + 8, low nibble = even column, for
   weights and int4 activations alike.
+* Tensor-wise input scale: a caller-supplied scalar a >= 0 multiplies x
+  before the rotation ([SD] review comments on docs/int8_convrot.md: inputs
+  whose scale is not 1 are scaled, then quantized; [RQ] "How was this patch
+  tested?": caller-provided zero tensor-wise scales follow eager
+  quantization). So a = 0 makes every row all-zero: s = 1, q = 0.
 * Epilogue: float32 ((float(acc) * s_m) * sw_n) (+ bias_n), each product
   rounded to float32, then round-to-nearest-even to bfloat16.
 """
@@ -118,9 +123,22 @@ def quantize_rowwise(y, bits: int):
     return q, s
 
 
-def rotate_quant_rowwise(x, G: int, bits: int, R=None):
-    """``quantize_and_rotate_rowwise``: rotation a1 then quantization a2-a3."""
-    return quantize_rowwise(rotate_groups(x, G, R), bits)
+def _check_input_scale(input_scale) -> float:
+    a = float(input_scale)
+    if not np.isfinite(a) or a < 0.0:
+        raise ValueError(f"input_scale={input_scale!r} must be finite and >= 0")
+    return a
+
+
+def rotate_quant_rowwise(x, G: int, bits: int, R=None, input_scale=1.0):
+    """``quantize_and_rotate_rowwise``: rotation a1 then quantization a2-a3.
+
+    ``input_scale`` is the caller's tensor-wise scale a: the rotated and
+    quantized matrix is that of a * x (the product taken in float64).
+    """
+    a = _check_input_scale(input_scale)
+    x = np.asarray(x, dtype=np.float64)
+    return quantize_rowwise(rotate_groups(a * x, G, R), bits)
 
 
 # --------------------------------------------------------------------------
@@ -219,14 +237,17 @@ def bf16_bits_to_f64(b) -> np.ndarray:
 # Composite paths
 # --------------------------------------------------------------------------
 
-def linear_w4a4(x, w_packed, w_scale, G: int, bias=None, R=None) -> dict:
+def linear_w4a4(x, w_packed, w_scale, G: int, bias=None, R=None, input_scale=1.0) -> dict:
     """ConvRot W4A4 linear: rotate + int4 quantize x, int matmul with the
     packed int4 weight, rowwise-scale epilogue to bf16.
+
+    With a tensor-wise ``input_scale`` a, the linear of a * x (the input is
+    scaled, then quantized; the output is not rescaled).
 
     Returns every intermediate: ``q`` (M, K) int, ``qa_packed`` (M, K/2) u8,
     ``s`` (M,) float32, ``acc`` (M, N) int64, ``y_f32`` and ``y_bits`` (bf16).
     """
-    q, s = rotate_quant_rowwise(x, G, 4, R)
+    q, s = rotate_quant_rowwise(x, G, 4, R, input_scale)
     acc = int_matmul(q, unpack_nibbles(w_packed))
     y32 = epilogue_rowwise(acc, s, w_scale, bias)
     return {"q": q, "qa_packed": pack_nibbles(q), "s": s, "acc": acc,

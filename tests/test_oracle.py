@@ -155,6 +155,72 @@ def test_all_zero_rows_give_unit_scale_and_zero_output():
     np.testing.assert_array_equal(r["y_f32"][2], bias)
 
 
+# ------------------------------------------------- tensor-wise input scale
+
+@pytest.mark.parametrize("G,bits", [(16, 4), (64, 8), (256, 4)])
+def test_zero_input_scale_quantizes_like_all_zero_rows(G, bits):
+    # a = 0 scales every row to zero: the positive-scale contract gives s = 1, q = 0
+    x = np.random.default_rng(11).standard_normal((5, 2 * G)) * 40
+    q, s = O.rotate_quant_rowwise(x, G, bits, input_scale=0.0)
+    assert np.all(q == 0)
+    np.testing.assert_array_equal(s, np.ones(5, dtype=np.float32))
+    bias = np.linspace(-1, 1, 7).astype(np.float32)
+    wp = np.random.default_rng(2).integers(0, 256, size=(7, G), dtype=np.uint8)
+    r = O.linear_w4a4(x, wp, np.full(7, 0.01, dtype=np.float32), G, bias=bias, input_scale=0.0)
+    np.testing.assert_array_equal(r["y_f32"], np.broadcast_to(bias, (5, 7)))
+
+
+@pytest.mark.parametrize("G,bits", [(16, 4), (64, 8)])
+def test_input_scale_multiplies_the_one_hot_amplitude(G, bits):
+    # one-hot 3 scaled by a = 5: every rotated entry is +-15 / sqrt(G), so
+    # s = 15 / sqrt(G) / qmax (dividing by a, or ignoring it, gives another s)
+    qmax = O.QMAX[bits]
+    i = G // 2 + 1
+    x = np.zeros((1, G))
+    x[0, i] = 3.0
+    q, s = O.rotate_quant_rowwise(x, G, bits, input_scale=5.0)
+    signs = np.array([(-1) ** bin(i & j).count("1") for j in range(G)])
+    np.testing.assert_array_equal(q[0], qmax * signs)
+    assert s[0] == np.float32(15.0 / np.sqrt(G) / qmax)
+
+
+@pytest.mark.parametrize("k", [-6, -1, 3, 10])
+def test_power_of_two_input_scale_keeps_codes_and_scales_s(k):
+    # scaling by 2^k is exact in binary floating point: the codes are those of
+    # x and every scale (and unbiased output) is 2^k times the unscaled one
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 128)) * rng.uniform(0.1, 10, size=(6, 1))
+    a = 2.0 ** k
+    for bits in (4, 8):
+        q1, s1 = O.rotate_quant_rowwise(x, 64, bits)
+        qa, sa = O.rotate_quant_rowwise(x, 64, bits, input_scale=a)
+        np.testing.assert_array_equal(qa, q1)
+        np.testing.assert_array_equal(sa, (s1 * np.float32(a)).astype(np.float32))
+    wp = rng.integers(0, 256, size=(9, 64), dtype=np.uint8)
+    sw = rng.uniform(0.005, 0.02, size=9).astype(np.float32)
+    r1 = O.linear_w4a4(x, wp, sw, 64)
+    ra = O.linear_w4a4(x, wp, sw, 64, input_scale=a)
+    np.testing.assert_array_equal(ra["acc"], r1["acc"])
+    np.testing.assert_array_equal(ra["y_f32"], (r1["y_f32"] * np.float32(a)).astype(np.float32))
+
+
+def test_general_input_scale_stays_within_half_a_step_of_the_scaled_rotation():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((10, 256))
+    a = 0.3712
+    y = O.rotate_groups(a * x, 64)
+    q, s = O.rotate_quant_rowwise(x, 64, 4, input_scale=a)
+    err = np.abs(q * s.astype(np.float64)[:, None] - y)
+    assert np.all(err <= 0.5 * s[:, None] * (1 + 1e-6))
+    np.testing.assert_array_equal(np.abs(q).max(axis=1), 7)
+
+
+@pytest.mark.parametrize("a", [-1.0, -0.0 - 1e-30, float("nan"), float("inf")])
+def test_input_scale_must_be_finite_and_nonnegative(a):
+    with pytest.raises(ValueError):
+        O.rotate_quant_rowwise(np.ones((1, 16)), 16, 4, input_scale=a)
+
+
 # -------------------------------------------------------------------- codec
 
 def test_codec_golden(golden_dir):
