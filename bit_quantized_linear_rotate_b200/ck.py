@@ -32,12 +32,14 @@ STATUS_NAMES = {0: "CK_OK", 1: "CK_ERR_INVALID_ARG", 2: "CK_ERR_UNSUPPORTED", 3:
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
 _int = ctypes.c_int
+_f32 = ctypes.c_float
 
 # name -> argument types (restype is ck_status = int unless listed below)
 SIGNATURES = {
     "ck_rotate_quant_rowwise": [_p, _int, _i64, _i64, _i64, _int, _int, _p, _p, _p],
     "ck_rotate_quant_rowwise_i8": [_p, _int, _i64, _i64, _i64, _int, _int, _p, _p, _p],
     "ck_rotate_quant_rowwise_r": [_p, _int, _i64, _i64, _i64, _int, _p, _int, _p, _p, _p],
+    "ck_rotate_quant_rowwise_scaled": [_p, _int, _i64, _i64, _i64, _int, _int, _f32, _p, _p, _p],
     "ck_gemm_w4a4": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemm_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_unpack_int4": [_p, _i64, _i64, _p, _p],
@@ -47,6 +49,8 @@ SIGNATURES = {
     "ck_linear_w4a4": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
     "ck_linear_w4a4_quantize": [_p, _int, _i64, _i64, _i64, _int, _p, ctypes.c_size_t, _p],
     "ck_linear_w4a4_matmul": [_i64, _i64, _i64, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
+    "ck_linear_w4a4_scaled": [_p, _int, _i64, _i64, _i64, _i64, _int, _f32, _p, _p, _p, _p, _p, ctypes.c_size_t,
+                              _p],
     "ck_linear_w4a4_static": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "ck_gemv_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemv_awq_w4a16": [_p, _int, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p],
@@ -176,6 +180,24 @@ def rotate_quant_rowwise_r(x, R, bits: int, q_out=None, scale_out=None, stream=N
     return q_out, scale_out
 
 
+def rotate_quant_rowwise_scaled(x, group_size: int, bits: int, input_scale: float, q_out=None,
+                                scale_out=None, stream=None):
+    """rotate_quant_rowwise of input_scale * x (a finite tensor-wise scale >= 0); same formats."""
+    _cuda(x)
+    M, K, ldx, x2 = _rows(x)
+    lead = tuple(x.shape[:-1])
+    if q_out is None:
+        q_out = torch.empty(lead + ((K // 2,) if bits == 4 else (K,)), device=x.device,
+                            dtype=torch.uint8 if bits == 4 else torch.int8)
+    if scale_out is None:
+        scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
+    _cuda(q_out, scale_out)
+    _check(lib.ck_rotate_quant_rowwise_scaled(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
+                                              float(input_scale), _ptr(q_out), _ptr(scale_out), _stream(stream)),
+           "ck_rotate_quant_rowwise_scaled")
+    return q_out, scale_out
+
+
 def unpack_int4(packed, out=None, stream=None):
     """(R, C/2) packed int4 -> (R, C) int8 with value u - 8."""
     _cuda(packed)
@@ -249,6 +271,24 @@ def linear_w4a4(x, w_packed, w_scale, group_size: int, bias=None, workspace=None
                               _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)),
            "ck_linear_w4a4")
+    return out
+
+
+def linear_w4a4_scaled(x, w_packed, w_scale, group_size: int, input_scale: float, bias=None, workspace=None,
+                       out=None, stream=None):
+    """linear_w4a4 of input_scale * x (a finite tensor-wise scale >= 0); the output is not rescaled."""
+    _cuda(x, w_packed, w_scale, bias)
+    M, K, ldx, x2 = _rows(x)
+    N = w_packed.shape[0]
+    ws_bytes = linear_w4a4_workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=x.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), device=x.device, dtype=torch.bfloat16)
+    _check(lib.ck_linear_w4a4_scaled(_ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size, float(input_scale),
+                                     _ptr(w_packed), _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "ck_linear_w4a4_scaled")
     return out
 
 

@@ -236,10 +236,15 @@ void launch_rq_g(const T* x, int64_t M, int K, int64_t ldx, int G, float rnorm, 
   launch_pdl(kern, dim3(persistent_grid<Tag>(kern, nt, smem, M)), dim3(nt), smem, st, x, M, K, ldx, G, rnorm, q, s, rs);
 }
 
+// in_scale: the caller's tensor-wise input scale a >= 0. The kernel's transform
+// is unnormalised (z = x H) and it scales z by rnorm both for the row amax and
+// for the codes, so rnorm = a / sqrt(G) yields the rotation and quantization of
+// a * x; a = 1 leaves rnorm = 1 / sqrt(G), exactly the unscaled launch. (G = 1
+// decides its codes from z and s alone and must have a = 1.)
 template <int QBITS, int STORE, typename T>
 void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, float* s, int32_t* rs, int nt,
-               cudaStream_t st) {
-  const float rnorm = (float)(1.0 / std::sqrt((double)G));
+               float in_scale, cudaStream_t st) {
+  const float rnorm = (float)((double)in_scale / std::sqrt((double)G));
   const T* xx = reinterpret_cast<const T*>(x);
   uint8_t* qq = reinterpret_cast<uint8_t*>(q);
   switch (G) {
@@ -253,24 +258,36 @@ void launch_rq(const void* x, int64_t M, int K, int64_t ldx, int G, void* q, flo
 
 template <typename T>
 void launch_rq_store(int bits, int store, const void* x, int64_t M, int K, int64_t ldx, int G, void* q,
-                     float* s, int32_t* rs, int nt, cudaStream_t st) {
+                     float* s, int32_t* rs, int nt, float a, cudaStream_t st) {
   using namespace ck::rq;
-  if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, K, ldx, G, q, s, rs, nt, st);
-  else if (store == STORE_INT8_PERM) launch_rq<4, STORE_INT8_PERM, T>(x, M, K, ldx, G, q, s, rs, nt, st);
-  else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, st);
-  else launch_rq<8, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, st);
+  if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
+  else if (store == STORE_INT8_PERM) launch_rq<4, STORE_INT8_PERM, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
+  else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
+  else launch_rq<8, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
 }
 
 // store: STORE_PACKED4 (bits 4), STORE_INT8 (codes as int8 bytes) or STORE_INT8_PERM
-// (bits 4, the linear's GEMM-ready activations with row sums in `rs`).
+// (bits 4, the linear's GEMM-ready activations with row sums in `rs`). in_scale:
+// the tensor-wise input scale, validated by the caller (finite, >= 0, 1 when G = 1).
 ck_status rotate_quant_impl(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int G,
-                            int bits, int store, void* q, float* s, int32_t* rs, cudaStream_t st) {
+                            int bits, int store, void* q, float* s, int32_t* rs, cudaStream_t st,
+                            float in_scale = 1.0f) {
   using namespace ck::rq;
   const int64_t nt = ((K + EPT - 1) / EPT + 31) / 32 * 32;
   if (nt > 512) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K=%lld too large (max 32768)", (long long)K);
-  if (xt == CK_BF16) launch_rq_store<__nv_bfloat16>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, st);
-  else launch_rq_store<__half>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, st);
+  if (xt == CK_BF16)
+    launch_rq_store<__nv_bfloat16>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, in_scale, st);
+  else launch_rq_store<__half>(bits, store, x, M, (int)K, ldx, G, q, s, rs, (int)nt, in_scale, st);
   return launch_status("rotate_quant");
+}
+
+// The tensor-wise input scale's contract: a finite a >= 0, and a = 1 when G = 1.
+ck_status check_input_scale(const char* who, float a, int group_size) {
+  if (!std::isfinite(a) || a < 0.0f)
+    return fail(CK_ERR_INVALID_ARG, "%s: input_scale=%g must be finite and >= 0", who, (double)a);
+  if (group_size == 1 && a != 1.0f)
+    return fail(CK_ERR_UNSUPPORTED, "%s: group_size 1 (no rotation) takes only input_scale 1", who);
+  return CK_OK;
 }
 
 ck_status check_gemm_shape(const char* who, int64_t M, int64_t K, int64_t N) {
@@ -412,26 +429,49 @@ const char* ck_last_error(void) { return g_last_error.c_str(); }
 
 const char* ck_version(void) { return "ck 0.1 (sm_100a)"; }
 
+}  // extern "C"
+
+namespace {
+
+ck_status rotate_quant_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                             int group_size, int bits, float in_scale, void* q_out, float* scale_out,
+                             void* stream) {
+  if (M < 0 || K <= 0) return fail(CK_ERR_INVALID_ARG, "%s: need M >= 0 and K > 0", who);
+  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "%s: unknown dtype", who);
+  if (bits != 4 && bits != 8) return fail(CK_ERR_INVALID_ARG, "%s: bits must be 4 or 8", who);
+  if (!is_pow2(group_size) || group_size > 256)
+    return fail(CK_ERR_UNSUPPORTED, "%s: group_size=%d must be a power of two <= 256", who, group_size);
+  ck_status r = check_input_scale(who, in_scale, group_size);
+  if (r != CK_OK) return r;
+  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "%s: K %% group_size != 0", who);
+  if (K % 8 != 0) return fail(CK_ERR_UNSUPPORTED, "%s: K must be a multiple of 8", who);
+  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "%s: ldx < K", who);
+  if (M == 0) return ok();
+  if (x == nullptr || q_out == nullptr || scale_out == nullptr)
+    return fail(CK_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "%s: x rows must be 16-byte aligned", who);
+  if (!aligned(q_out, 16) || !aligned(scale_out, 4)) return fail(CK_ERR_INVALID_ARG, "%s: misaligned output", who);
+  if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "%s: M too large", who);
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits,
+                           bits == 4 ? ck::rq::STORE_PACKED4 : ck::rq::STORE_INT8, q_out, scale_out,
+                           nullptr, S(stream), in_scale);
+}
+
+}  // namespace
+
+extern "C" {
+
 ck_status ck_rotate_quant_rowwise(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
                                   int group_size, int bits, void* q_out, float* scale_out,
                                   void* stream) {
-  if (M < 0 || K <= 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant: need M >= 0 and K > 0");
-  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "rotate_quant: unknown dtype");
-  if (bits != 4 && bits != 8) return fail(CK_ERR_INVALID_ARG, "rotate_quant: bits must be 4 or 8");
-  if (!is_pow2(group_size) || group_size > 256)
-    return fail(CK_ERR_UNSUPPORTED, "rotate_quant: group_size=%d must be a power of two <= 256", group_size);
-  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant: K %% group_size != 0");
-  if (K % 8 != 0) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: K must be a multiple of 8");
-  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "rotate_quant: ldx < K");
-  if (M == 0) return ok();
-  if (x == nullptr || q_out == nullptr || scale_out == nullptr)
-    return fail(CK_ERR_INVALID_ARG, "rotate_quant: null pointer");
-  if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "rotate_quant: x rows must be 16-byte aligned");
-  if (!aligned(q_out, 16) || !aligned(scale_out, 4)) return fail(CK_ERR_INVALID_ARG, "rotate_quant: misaligned output");
-  if (M > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "rotate_quant: M too large");
-  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits,
-                           bits == 4 ? ck::rq::STORE_PACKED4 : ck::rq::STORE_INT8, q_out, scale_out,
-                           nullptr, S(stream));
+  return rotate_quant_entry("rotate_quant", x, xt, M, K, ldx, group_size, bits, 1.0f, q_out, scale_out, stream);
+}
+
+ck_status ck_rotate_quant_rowwise_scaled(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                         int group_size, int bits, float input_scale, void* q_out,
+                                         float* scale_out, void* stream) {
+  return rotate_quant_entry("rotate_quant_scaled", x, xt, M, K, ldx, group_size, bits, input_scale, q_out,
+                            scale_out, stream);
 }
 
 ck_status ck_rotate_quant_rowwise_i8(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
@@ -556,21 +596,37 @@ size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K) {
   return linear_q_bytes(M, K) + align256((size_t)M * sizeof(float)) + (size_t)M * sizeof(int32_t);
 }
 
-ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int group_size,
-                                  void* workspace, size_t ws_bytes, void* stream) {
-  ck_status r = check_gemm_shape("linear_w4a4_quantize", M, K, 1);
+}  // extern "C"
+
+namespace {
+
+ck_status linear_quantize_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                int group_size, float in_scale, void* workspace, size_t ws_bytes, void* stream) {
+  ck_status r = check_gemm_shape(who, M, K, 1);
   if (r != CK_OK) return r;
-  if ((r = check_linear_workspace("linear_w4a4_quantize", M, K, workspace, ws_bytes)) != CK_OK) return r;
-  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: unknown dtype");
+  if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
+  if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "%s: unknown dtype", who);
   if (!is_pow2(group_size) || group_size > 256)
-    return fail(CK_ERR_UNSUPPORTED, "linear_w4a4_quantize: group_size=%d must be a power of two <= 256", group_size);
-  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: K %% group_size != 0");
-  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: ldx < K");
-  if (x == nullptr) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: null pointer");
-  if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_quantize: x rows must be 16-byte aligned");
+    return fail(CK_ERR_UNSUPPORTED, "%s: group_size=%d must be a power of two <= 256", who, group_size);
+  if ((r = check_input_scale(who, in_scale, group_size)) != CK_OK) return r;
+  if (K % group_size != 0) return fail(CK_ERR_INVALID_ARG, "%s: K %% group_size != 0", who);
+  if (ldx < K) return fail(CK_ERR_INVALID_ARG, "%s: ldx < K", who);
+  if (x == nullptr) return fail(CK_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "%s: x rows must be 16-byte aligned", who);
   LinearWs ws = linear_ws(workspace, M, K);
   const int store = linear_small_m(M, K) ? ck::rq::STORE_INT8 : ck::rq::STORE_INT8_PERM;
-  return rotate_quant_impl(x, xt, M, K, ldx, group_size, 4, store, ws.q, ws.scale, ws.rowsum, S(stream));
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, 4, store, ws.q, ws.scale, ws.rowsum, S(stream),
+                           in_scale);
+}
+
+}  // namespace
+
+extern "C" {
+
+ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int group_size,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  return linear_quantize_entry("linear_w4a4_quantize", x, xt, M, K, ldx, group_size, 1.0f, workspace, ws_bytes,
+                               stream);
 }
 
 ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
@@ -596,21 +652,44 @@ ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* 
       ws.q, M, K, N, w_packed, ws.scale, ws.rowsum, w_scale, bias, y, S(stream));
 }
 
+}  // extern "C"
+
+namespace {
+
+ck_status linear_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
+                       int group_size, float in_scale, const uint8_t* w_packed, const uint16_t* w_scale,
+                       const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+  ck_status r = check_gemm_shape(who, M, K, N);
+  if (r != CK_OK) return r;
+  // validate both phases before enqueuing either
+  if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
+  if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "%s: weights must be 16-byte aligned", who);
+  if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
+  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, in_scale, workspace, ws_bytes, stream);
+  if (r != CK_OK) return r;
+  return ck_linear_w4a4_matmul(M, K, N, w_packed, w_scale, bias, y, workspace, ws_bytes, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
 ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
                          int group_size, const uint8_t* w_packed, const uint16_t* w_scale,
                          const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes,
                          void* stream) {
-  ck_status r = check_gemm_shape("linear_w4a4", M, K, N);
-  if (r != CK_OK) return r;
-  // validate both phases before enqueuing either
-  if ((r = check_linear_workspace("linear_w4a4", M, K, workspace, ws_bytes)) != CK_OK) return r;
-  if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "linear_w4a4: null pointer");
-  if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "linear_w4a4: weights must be 16-byte aligned");
-  if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
-    return fail(CK_ERR_INVALID_ARG, "linear_w4a4: misaligned scale, bias or output");
-  r = ck_linear_w4a4_quantize(x, xt, M, K, ldx, group_size, workspace, ws_bytes, stream);
-  if (r != CK_OK) return r;
-  return ck_linear_w4a4_matmul(M, K, N, w_packed, w_scale, bias, y, workspace, ws_bytes, stream);
+  return linear_entry("linear_w4a4", x, xt, M, K, N, ldx, group_size, 1.0f, w_packed, w_scale, bias, y,
+                      workspace, ws_bytes, stream);
+}
+
+ck_status ck_linear_w4a4_scaled(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
+                                int group_size, float input_scale, const uint8_t* w_packed,
+                                const uint16_t* w_scale, const uint16_t* bias, uint16_t* y, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  return linear_entry("linear_w4a4_scaled", x, xt, M, K, N, ldx, group_size, input_scale, w_packed, w_scale,
+                      bias, y, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -97,6 +97,31 @@ ck_status ck_rotate_quant_rowwise_r(const void* x, ck_dtype xt, int64_t M, int64
                                     float* scale_out, void* stream);
 
 /*
+ * ck_rotate_quant_rowwise of a * x, for a caller-supplied tensor-wise input
+ * scale a. Two passages touch this scale:
+ *   - comfy-kitchen PR #155, "How was this patch tested?": caller-provided
+ *     zero tensor-wise scales follow eager quantization;
+ *   - stable-diffusion.cpp PR #2276, review comments on docs/int8_convrot.md:
+ *     inputs whose scale is not 1 are scaled, then quantized.
+ * Neither gives a formula. The reading taken is that a multiplies x before
+ * the rotation:
+ *   y_g = (a x_g) . H_G / sqrt(G), then s_m and q as for ck_rotate_quant_rowwise.
+ * a = 0 makes every row all-zero: s_m = 1 and q = 0. a = 1 gives exactly the
+ * results of ck_rotate_quant_rowwise. Same kernel and speed: the scale folds
+ * into the transform's normalisation.
+ * input_scale : host value, finite and >= 0 (else CK_ERR_INVALID_ARG). The
+ *               scaled rows must stay in fp32's normal range: a row whose
+ *               nonzero scale s_m would fall below 2^-126, or overflow, gets
+ *               unspecified codes.
+ * group_size  : a power of two <= 256. 1 (no rotation) is accepted only
+ *               with a = 1 (CK_ERR_UNSUPPORTED otherwise).
+ * Other arguments, formats and errors as for ck_rotate_quant_rowwise.
+ */
+ck_status ck_rotate_quant_rowwise_scaled(const void* x, ck_dtype xt, int64_t M, int64_t K,
+                                         int64_t ldx, int group_size, int bits, float input_scale,
+                                         void* q_out, float* scale_out, void* stream);
+
+/*
  * Integer matmul of packed int4 activations with packed int4 weights, int32
  * accumulation on the tcgen05 tensor cores, and the rowwise-scale epilogue
  * (the "EpiRowwise" of comfy-kitchen PR #182, Description):
@@ -185,6 +210,22 @@ ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t
 ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed,
                                 const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
                                 const void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * ck_linear_w4a4 of a * x, for a tensor-wise input scale a. It follows the
+ * reading of ck_rotate_quant_rowwise_scaled. stable-diffusion.cpp PR #2276,
+ * review comments on docs/int8_convrot.md: ggml_mul_mat_w4_convrot scales
+ * inputs whose scale is not 1, then quantizes them. y is the linear of a * x
+ * and is not divided by a afterwards. a = 1 gives exactly ck_linear_w4a4's
+ * results, and a = 0 gives y = bias (or 0) in every row.
+ * input_scale : as for ck_rotate_quant_rowwise_scaled.
+ * Other arguments, the workspace and its size as for ck_linear_w4a4.
+ */
+ck_status ck_linear_w4a4_scaled(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N,
+                                int64_t ldx, int group_size, float input_scale,
+                                const uint8_t* w_packed, const uint16_t* w_scale,
+                                const uint16_t* bias, uint16_t* y, void* workspace,
+                                size_t ws_bytes, void* stream);
 
 /* Size of the scratch built into the library for ck_linear_w4a4_static: 32 MiB per device. */
 #define CK_LINEAR_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)

@@ -143,6 +143,42 @@ def test_general_rotation_validation(ck):
     assert call(M=0, x=None, R=None, q=None, s=None) == ck.CK_OK
 
 
+@pytest.mark.parametrize("a", [float("nan"), float("inf"), -1.0, -1e-30])
+def test_input_scale_must_be_finite_and_nonnegative(ck, a):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    assert L.ck_rotate_quant_rowwise_scaled(P(1 << 20), 0, 4, 64, 64, 64, 4, a, P(1 << 21), P(1 << 22),
+                                            None) == ck.CK_ERR_INVALID_ARG
+    assert "input_scale" in ck.last_error()
+    ws = ck.linear_w4a4_workspace_bytes(8, 64)
+    assert L.ck_linear_w4a4_scaled(P(1 << 20), 0, 8, 64, 8, 64, 64, a, P(1 << 20), P(1 << 20), None,
+                                   P(1 << 20), P(1 << 21), ws, None) == ck.CK_ERR_INVALID_ARG
+
+
+def test_input_scale_other_checks(ck):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    def rq(**kw):
+        a = dict(x=P(1 << 20), M=4, K=64, G=64, bits=4, a=0.5)
+        a.update(kw)
+        return L.ck_rotate_quant_rowwise_scaled(a["x"], 0, a["M"], a["K"], a["K"], a["G"], a["bits"], a["a"],
+                                                P(1 << 21), P(1 << 22), None)
+    assert rq(G=1, a=2.0) == ck.CK_ERR_UNSUPPORTED        # no rotation: only a = 1
+    assert rq(G=1, a=1.0, M=0) == ck.CK_OK
+    assert rq(M=0, a=0.0) == ck.CK_OK                     # empty input: no-op
+    assert rq(G=48) == ck.CK_ERR_UNSUPPORTED
+    assert rq(bits=5) == ck.CK_ERR_INVALID_ARG
+    assert rq(x=None) == ck.CK_ERR_INVALID_ARG
+    assert rq(x=P((1 << 20) + 2)) == ck.CK_ERR_INVALID_ARG
+    ws = ck.linear_w4a4_workspace_bytes(8, 64)
+    lin = lambda G, a, ws_bytes=ws: L.ck_linear_w4a4_scaled(P(1 << 20), 0, 8, 64, 8, 64, G, a, P(1 << 20),
+                                                            P(1 << 20), None, P(1 << 20), P(1 << 21), ws_bytes,
+                                                            None)
+    assert lin(1, 3.0) == ck.CK_ERR_UNSUPPORTED
+    assert lin(48, 1.0) == ck.CK_ERR_UNSUPPORTED
+    assert lin(64, 1.0, ws - 1) == ck.CK_ERR_INVALID_ARG
+
+
 def test_selftest_timeout_range_is_validated(ck):
     assert ck.lib.ck_selftest_bounded_wait(10, None) == ck.CK_ERR_INVALID_ARG
     assert ck.lib.ck_selftest_bounded_wait(10 ** 10, None) == ck.CK_ERR_INVALID_ARG

@@ -273,6 +273,70 @@ def test_linear_w4a4_matches_oracle(ck, M, K, N, G, bias, dtype):
     assert_out_close(to_np_f64(y), O.bf16_bits_to_f64(r["y_bits"]))
 
 
+# ------------------------------------------------- tensor-wise input scale
+
+@pytest.mark.parametrize("G,bits,dtype,a", [
+    (16, 4, torch.bfloat16, 0.37), (64, 8, torch.float16, 5.5), (256, 4, torch.bfloat16, 1e-3),
+    (64, 4, torch.float16, 3.0e4), (32, 8, torch.bfloat16, 0.71), (64, 4, torch.bfloat16, 0.0),
+])
+def test_rotate_quant_scaled_matches_oracle(ck, G, bits, dtype, a):
+    M, K = 37, 768
+    xf = _rand_x(M, K + 64, seed=G + bits, dtype=dtype, outliers=6)
+    x = xf.to(DEV)[:, :K]
+    q, s = ck.rotate_quant_rowwise_scaled(x, G, bits, a)
+    torch.cuda.synchronize()
+    q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf[:, :K]), G, bits, input_scale=a)
+    q_gpu = unpack_codes(q) if bits == 4 else q.cpu().numpy()
+    if a == 0.0:
+        assert np.all(s.cpu().numpy() == 1.0) and np.all(q_gpu == 0)
+    assert_scales_close(s.cpu().numpy(), s_ref)
+    assert_codes_close(q_gpu, q_ref)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_rotate_quant_scaled_by_powers_of_two_is_exact(ck, bits):
+    # a = 1 is the unscaled call bit for bit; a = 2^k keeps every code and
+    # multiplies every scale by 2^k exactly (each step is exact in binary fp)
+    M, K, G = 300, 1024, 64
+    x = _rand_x(M, K, seed=9, outliers=10).to(DEV)
+    q1, s1 = ck.rotate_quant_rowwise(x, G, bits)
+    for a in (1.0, 0.125, 64.0):
+        qa, sa = ck.rotate_quant_rowwise_scaled(x, G, bits, a)
+        torch.cuda.synchronize()
+        assert torch.equal(qa, q1)
+        assert torch.equal(sa, s1 * a)
+
+
+@pytest.mark.parametrize("M,K,N,G,bias,dtype,a", [
+    (300, 1024, 520, 64, True, torch.bfloat16, 0.37),
+    (129, 768, 260, 256, False, torch.float16, 12.0),
+    (32, 3840, 520, 64, True, torch.bfloat16, 2.5),        # small-batch route
+    (200, 512, 300, 16, True, torch.bfloat16, 0.0),
+])
+def test_linear_w4a4_scaled_matches_oracle(ck, M, K, N, G, bias, dtype, a):
+    d = WL.small_linear_inputs(M, K, N, seed=M + N, n_outlier_cols=K // 100, dtype=dtype, with_bias=bias)
+    b = d.get("bias")
+    y = ck.linear_w4a4_scaled(d["x"].to(DEV), d["w_packed"].to(DEV), d["w_scale"].to(DEV), G, a,
+                              bias=None if b is None else b.to(DEV))
+    r = O.linear_w4a4(to_np_f64(d["x"]), d["w_packed"].numpy(), to_np_f64(d["w_scale"]), G,
+                      bias=None if b is None else to_np_f64(b), input_scale=a)
+    if a == 0.0:
+        # every row quantizes to zero codes: y is the bias, exactly
+        expect = b.expand(M, N) if b is not None else torch.zeros(M, N, dtype=torch.bfloat16)
+        assert torch.equal(y.cpu(), expect.to(torch.bfloat16))
+    assert_out_close(to_np_f64(y), O.bf16_bits_to_f64(r["y_bits"]))
+
+
+def test_linear_w4a4_scaled_by_one_is_the_unscaled_call(ck):
+    for M in (300, 32):
+        d = WL.small_linear_inputs(M, 1024, 264, seed=3, n_outlier_cols=10, with_bias=True)
+        args = (d["x"].to(DEV), d["w_packed"].to(DEV), d["w_scale"].to(DEV), 64)
+        y1 = ck.linear_w4a4(*args, bias=d["bias"].to(DEV))
+        ya = ck.linear_w4a4_scaled(*args, 1.0, bias=d["bias"].to(DEV))
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_tensor_bits(ya), bf16_tensor_bits(y1))
+
+
 def _a256(v):
     return (v + 255) // 256 * 256
 
