@@ -432,6 +432,14 @@ def time_other_configs(ck, dev, peaks):
         out[f"rotate_quant_M{M}_K{K}_G{G}_int{bits}"] = {
             "us": round(ms * 1e3, 2), "GBps": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "copies": R}
+        if (M, K, G) == (8192, 3840, 64) and bits == 8:
+            # the linear's own quantize phase (permuted codes + row sums), back to back
+            ws = torch.empty(ck.linear_w4a4_workspace_bytes(M, K), device=dev, dtype=torch.uint8)
+            ms = time_rotating(lambda c: ck.linear_w4a4_quantize(xs[c], G, ws), R, 100, 5)
+            nbytes = M * K * 2 + M * K + 8 * M
+            out[f"linear_quantize_M{M}_K{K}_G{G}"] = {
+                "us": round(ms * 1e3, 2), "GBps": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "copies": R}
         del xs
     return out
 
