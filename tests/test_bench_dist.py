@@ -67,6 +67,26 @@ def test_two_rank_barrier_and_max_over_ranks():
     assert got[1][2] == ""          # rank 1 printed nothing
 
 
+def test_reference_arm_prints_one_contract_line_on_rank_zero():
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.run_reference(type("A", (), {"warmup": 0, "steps": 1, "cpu_rows": 16})(), 1, 0)
+    lines = [l for l in out.getvalue().splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert "workload" in d["config"]
+
+
 def test_value_is_aggregate_units_over_slowest_rank():
     # value = 2*M*N*K*steps*world / slowest time, i.e. per-rank work is fixed (weak scaling)
     sys.path.insert(0, ROOT)
