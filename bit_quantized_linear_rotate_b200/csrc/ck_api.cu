@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -135,17 +136,31 @@ ck::gstream::Layout stream_layout_m8(int stage_bytes, int misc_bytes);
 // the runtime reserves per CTA) fit in an SM's 228 KB.
 constexpr int kStreamSmemMax = 112 * 1024;
 
-// Raises a kernel's dynamic shared-memory limit to `bytes` once per device
-// (cached per kernel instantiation through Tag; the largest value set wins).
+// The host-side caches below hold per-device facts (a kernel attribute that was
+// set, an occupancy, an SM count). Each entry is an atomic, so calls from
+// several host threads may race to fill one; they compute the same value, and
+// setting a kernel attribute twice to the same value is harmless.
+constexpr int kMaxDevices = 64;
+
+// The current device, or -1 when it cannot be read or is beyond the caches.
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+// Raises a stream kernel's dynamic shared-memory limit to kStreamSmemMax (the
+// most any of its launches asks for, `bytes` <= kStreamSmemMax) once per
+// device, cached per kernel instantiation through Tag.
 template <typename Tag, typename KernelT>
 cudaError_t set_smem_max(KernelT kern, int bytes) {
-  static int done[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
-  if (done[dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
-  if (e == cudaSuccess) done[dev] = kStreamSmemMax;
+  static std::atomic<bool> done[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (bytes > kStreamSmemMax) return cudaErrorInvalidValue;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
   return e;
 }
 
@@ -183,46 +198,57 @@ ck::gstream::Layout stream_layout(int stage_bytes, int misc_bytes) {
 
 // ------------------------------------------------------------------ kernels
 
-// One cache per kernel instantiation (the Tag template argument), per device.
+// Sets a kernel's dynamic shared-memory limit to `bytes` (the fixed size of
+// all its launches) once per device, cached per kernel instantiation (Tag).
 template <typename Tag, typename KernelT>
 ck_status ensure_smem_attr(KernelT kernel, size_t bytes) {
-  static bool done[64] = {false};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(CK_ERR_CUDA, "cudaGetDevice failed");
-  if (!done[dev]) {
+  static std::atomic<bool> done[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return fail(CK_ERR_CUDA, "cudaGetDevice failed");
+  if (!done[dev].load(std::memory_order_acquire)) {
     const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return fail(CK_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
   }
   return CK_OK;
 }
 
 int sm_count() {
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
-// Persistent grid: as many CTAs of `nt` threads (and `smem` dynamic bytes) as
-// are co-resident (cached per kernel instantiation, through Tag, and nt).
+// Persistent grid: as many CTAs of `nt` threads (a multiple of 32, at most
+// 1024) and `smem` dynamic bytes as are co-resident, at most `work`. The
+// kernel's dynamic shared-memory limit is raised once per device to
+// `smem_max`, the most ANY launch of this kernel asks for: raising it to each
+// launch's own size would lower it again for a smaller launch and make a later
+// larger one fail. The occupancy is cached per kernel instantiation (Tag),
+// device and nt.
 template <typename Tag, typename KernelT>
-unsigned persistent_grid(KernelT kern, int nt, size_t smem, int64_t work) {
-  static int cache_nt[64] = {0}, cache_blocks[64] = {0};
-  const int slot = (nt / 32) & 63;
-  int blocks = 0;
-  if (cache_nt[slot] == nt) {
-    blocks = cache_blocks[slot];
-  } else {
-    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, nt, smem) != cudaSuccess || blocks <= 0) blocks = 1;
-    cache_blocks[slot] = blocks;
-    cache_nt[slot] = nt;
+unsigned persistent_grid(KernelT kern, int nt, size_t smem, size_t smem_max, int64_t work) {
+  static std::atomic<bool> limit_set[kMaxDevices];
+  static std::atomic<int> cache[kMaxDevices][32];   // [dev][nt / 32 - 1]: CTAs per SM, 0 = not known
+  const int dev = current_device();
+  const int slot = nt / 32 - 1;
+  const bool cached = dev >= 0 && nt % 32 == 0 && slot >= 0 && slot < 32;
+  if (smem_max > 48 * 1024 && !(cached && limit_set[dev].load(std::memory_order_acquire))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) == cudaSuccess &&
+        cached)
+      limit_set[dev].store(true, std::memory_order_release);
+  }
+  int blocks = cached ? cache[dev][slot].load(std::memory_order_relaxed) : 0;
+  if (blocks <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, nt, smem) != cudaSuccess || blocks <= 0)
+      blocks = 1;
+    if (cached) cache[dev][slot].store(blocks, std::memory_order_relaxed);
   }
   return (unsigned)std::min<int64_t>(work, (int64_t)blocks * sm_count());
 }
@@ -232,8 +258,10 @@ void launch_rq_g(const T* x, int64_t M, int K, int64_t ldx, int G, float rnorm, 
                  int nt, cudaStream_t st) {
   auto kern = ck::rq::rotate_quant_kernel<QBITS, STORE, GT, T>;
   const size_t smem = (size_t)(nt / 32) * 32 * ck::rq::CPT * 16;   // one transpose buffer per warp
+  const size_t smem_max = (size_t)512 * ck::rq::CPT * 16;            // at the most threads a launch takes
   struct Tag {};
-  launch_pdl(kern, dim3(persistent_grid<Tag>(kern, nt, smem, M)), dim3(nt), smem, st, x, M, K, ldx, G, rnorm, q, s, rs);
+  launch_pdl(kern, dim3(persistent_grid<Tag>(kern, nt, smem, smem_max, M)), dim3(nt), smem, st, x, M, K, ldx, G,
+             rnorm, q, s, rs);
 }
 
 // in_scale: the caller's tensor-wise input scale a >= 0. The kernel's transform
@@ -303,10 +331,11 @@ ck_status check_gemm_shape(const char* who, int64_t M, int64_t K, int64_t N) {
 // Largest number of CTA pairs of this kernel that are co-resident on the device (cached per device).
 template <typename Tag, typename KernelT>
 ck_status max_pairs(KernelT kernel, size_t smem, int* out) {
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(CK_ERR_CUDA, "cudaGetDevice failed");
-  if (cache[dev] == 0) {
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return fail(CK_ERR_CUDA, "cudaGetDevice failed");
+  int pairs = cache[dev].load(std::memory_order_relaxed);
+  if (pairs == 0) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -321,9 +350,10 @@ ck_status max_pairs(KernelT kernel, size_t smem, int* out) {
     int n = 0;
     const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
     if (e != cudaSuccess || n <= 0) return fail(CK_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s (%d)", cudaGetErrorString(e), n);
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
+    pairs = n;
   }
-  *out = cache[dev];
+  *out = pairs;
   return CK_OK;
 }
 

@@ -141,6 +141,18 @@ def test_rotate_quant_long_rows(ck, M, K):
     assert_codes_close(unpack_codes(q.cpu()[rows]), q_ref)
 
 
+def test_rotate_quant_alternating_row_lengths(ck):
+    # launches of one kernel with different dynamic shared memory (64 KB at
+    # K = 32768, 56 KB at K = 28672), a larger one after a smaller one
+    for K in (32768, 28672, 32768, 24576, 32768):
+        xf = _rand_x(3, K, seed=K + 1, outliers=K // 100)
+        q, s = ck.rotate_quant_rowwise(xf.to(DEV), 64, 4)
+        torch.cuda.synchronize()
+        q_ref, s_ref = O.rotate_quant_rowwise(to_np_f64(xf), 64, 4)
+        assert_scales_close(s.cpu().numpy(), s_ref)
+        assert_codes_close(unpack_codes(q), q_ref)
+
+
 def test_rotate_quant_mlp_down_G16_full(ck):
     w = WL.LINEAR_MLP_DOWN
     x = WL.linear_inputs(w)["x"]
