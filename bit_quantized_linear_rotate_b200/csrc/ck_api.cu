@@ -180,7 +180,11 @@ ck::gstream::Layout stream_layout_m8(int stage_bytes, int misc_bytes) {
 
 // Shared-memory layout of a streaming GEMV: as many stages as fit in half of
 // an SM's shared memory, so that the next call's CTA can be resident (and
-// streaming its first tiles) while this one runs.
+// streaming its first tiles) while this one runs. The per-CTA slices of the
+// weight scales and bias (misc_bytes) grow with N / SMs; when they leave room
+// for fewer than two stages (L.ns < 2, possibly negative) the streaming
+// kernel cannot run and the caller takes the general kernel. The same holds
+// for stream_layout_m8.
 ck::gstream::Layout stream_layout(int stage_bytes, int misc_bytes) {
   using namespace ck::gstream;
   Layout L;
@@ -542,13 +546,16 @@ ck_status ck_rotate_quant_rowwise_r(const void* x, ck_dtype xt, int64_t M, int64
   if (!aligned(x, 2) || !aligned(R, 4) || !aligned(scale_out, 4))
     return fail(CK_ERR_INVALID_ARG, "rotate_quant_rowwise_r: misaligned pointer");
   const size_t smem = 2 * (size_t)K * sizeof(float);
+  const size_t smem_max = 2 * (size_t)16384 * sizeof(float);   // K <= 16384: the limit, set once per device
   const unsigned grid = (unsigned)std::min<int64_t>(M, 8 * (int64_t)sm_count());
   cudaError_t e = cudaSuccess;
+  ck_status r = CK_OK;
 #define CK_RQG(T, B)                                                                                 \
   {                                                                                                  \
     auto kern = ck::rqg::rotate_quant_general_kernel<T, B>;                                          \
-    if (smem > 48 * 1024) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-    if (e == cudaSuccess)                                                                            \
+    struct Tag {};                                                                                   \
+    r = ensure_smem_attr<Tag>(kern, smem_max);                                                       \
+    if (r == CK_OK)                                                                                  \
       e = launch_pdl(kern, dim3(grid), dim3(ck::rqg::kThreads), smem, S(stream), reinterpret_cast<const T*>(x), M, \
                      (int)K, ldx, group_size, R, reinterpret_cast<uint8_t*>(q_out), scale_out);       \
   }
@@ -558,6 +565,7 @@ ck_status ck_rotate_quant_rowwise_r(const void* x, ck_dtype xt, int64_t M, int64
     if (bits == 4) CK_RQG(__half, 4) else CK_RQG(__half, 8)
   }
 #undef CK_RQG
+  if (r != CK_OK) return r;
   if (e != cudaSuccess) return fail(CK_ERR_CUDA, "rotate_quant_rowwise_r: %s", cudaGetErrorString(e));
   return launch_status("rotate_quant_rowwise_r");
 }
@@ -828,22 +836,24 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
     ck_status r = make_tmap_wtile(&tw, w_packed, (uint64_t)N, (uint64_t)K, 16);
     if (r != CK_OK) return r;
     sp.L = stream_layout_m8((int)(16 * (K / 2)), kCons * 8 * 4 + 2 * 16 * tpc * 4 + 16);
-    const int nchunk = (int)(K / 128), cpw = (nchunk + kCons - 1) / kCons;
-    cudaError_t e;
+    if (sp.L.ns >= 2) {   // else too many tiles per CTA for the ring: general kernel
+      const int nchunk = (int)(K / 128), cpw = (nchunk + kCons - 1) / kCons;
+      cudaError_t e;
 #define CK_W4A8_STREAM_M8(CPW)                                                                   \
-    {                                                                                            \
-      auto kern = w4a8_stream_m8_kernel<CPW>;                                                    \
-      struct Tag {};                                                                             \
-      e = set_smem_max<Tag>(kern, sp.L.total);                                                   \
-      if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), sp.L.total, S(stream), tw, sp); \
-    }
-    if (cpw <= 1) CK_W4A8_STREAM_M8(1)
-    else if (cpw == 2) CK_W4A8_STREAM_M8(2)
-    else if (cpw == 3) CK_W4A8_STREAM_M8(3)
-    else CK_W4A8_STREAM_M8(4)
+      {                                                                                            \
+        auto kern = w4a8_stream_m8_kernel<CPW>;                                                    \
+        struct Tag {};                                                                             \
+        e = set_smem_max<Tag>(kern, sp.L.total);                                                   \
+        if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), sp.L.total, S(stream), tw, sp); \
+      }
+      if (cpw <= 1) CK_W4A8_STREAM_M8(1)
+      else if (cpw == 2) CK_W4A8_STREAM_M8(2)
+      else if (cpw == 3) CK_W4A8_STREAM_M8(3)
+      else CK_W4A8_STREAM_M8(4)
 #undef CK_W4A8_STREAM_M8
-    if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
-    return launch_status("gemv_w4a8");
+      if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
+      return launch_status("gemv_w4a8");
+    }
   }
   if (K <= 4096) {
     // streaming path: 8-row weight tiles through a shared-memory ring, one CTA per SM
@@ -856,22 +866,24 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
     const int tpc = (sp.ntiles + grid - 1) / grid;
     sp.srow = (int)(K / 2) + 64;
     sp.L = stream_layout(8 * sp.srow, kCons * 16 * 4 + 2 * 8 * tpc * 4 + 16);
-    const int nchunk = (int)(K / 128), cpw = (nchunk + kCons - 1) / kCons;
-    cudaError_t e;
+    if (sp.L.ns >= 2) {   // else too many tiles per CTA for the ring: general kernel
+      const int nchunk = (int)(K / 128), cpw = (nchunk + kCons - 1) / kCons;
+      cudaError_t e;
 #define CK_W4A8_STREAM(CPW)                                                                      \
-    {                                                                                            \
-      auto kern = w4a8_stream_kernel<CPW>;                                                       \
-      struct Tag {};                                                                             \
-      e = set_smem_max<Tag>(kern, sp.L.total);                                                   \
-      if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), sp.L.total, S(stream), sp); \
-    }
-    if (cpw <= 1) CK_W4A8_STREAM(1)
-    else if (cpw == 2) CK_W4A8_STREAM(2)
-    else if (cpw == 3) CK_W4A8_STREAM(3)
-    else CK_W4A8_STREAM(4)
+      {                                                                                            \
+        auto kern = w4a8_stream_kernel<CPW>;                                                       \
+        struct Tag {};                                                                             \
+        e = set_smem_max<Tag>(kern, sp.L.total);                                                   \
+        if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), sp.L.total, S(stream), sp); \
+      }
+      if (cpw <= 1) CK_W4A8_STREAM(1)
+      else if (cpw == 2) CK_W4A8_STREAM(2)
+      else if (cpw == 3) CK_W4A8_STREAM(3)
+      else CK_W4A8_STREAM(4)
 #undef CK_W4A8_STREAM
-    if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
-    return launch_status("gemv_w4a8");
+      if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
+      return launch_status("gemv_w4a8");
+    }
   }
   const unsigned grid = (unsigned)((N + ck::w4a8::kRows - 1) / ck::w4a8::kRows);
   if (M <= 8)
@@ -920,29 +932,31 @@ ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, in
     const int grid = std::min(ap.ntiles, sm_count());
     const int tpc = (ap.ntiles + grid - 1) / grid;
     ap.L = stream_layout(ap.w_bytes + 2 * ap.sz_stride, 16 * tpc * 4 + 16);
-    const int nsub = (int)(K / 64), spw = (nsub + kCons - 1) / kCons;
-    cudaError_t e = cudaSuccess;
+    if (ap.L.ns >= 2) {   // else too many tiles per CTA for the ring: general kernel
+      const int nsub = (int)(K / 64), spw = (nsub + kCons - 1) / kCons;
+      cudaError_t e = cudaSuccess;
 #define CK_AWQ_STREAM(T, SPW)                                                                    \
-    {                                                                                            \
-      auto kern = awq_stream_kernel<T, SPW>;                                                     \
-      struct Tag {};                                                                             \
-      e = set_smem_max<Tag>(kern, ap.L.total);                                                   \
-      if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), ap.L.total, S(stream), ts, tz, ap); \
-    }
-    if (dt == CK_BF16) {
-      if (spw <= 2) CK_AWQ_STREAM(__nv_bfloat16, 2)
-      else if (spw <= 4) CK_AWQ_STREAM(__nv_bfloat16, 4)
-      else if (spw <= 6) CK_AWQ_STREAM(__nv_bfloat16, 6)
-      else CK_AWQ_STREAM(__nv_bfloat16, 8)
-    } else {
-      if (spw <= 2) CK_AWQ_STREAM(__half, 2)
-      else if (spw <= 4) CK_AWQ_STREAM(__half, 4)
-      else if (spw <= 6) CK_AWQ_STREAM(__half, 6)
-      else CK_AWQ_STREAM(__half, 8)
-    }
+      {                                                                                            \
+        auto kern = awq_stream_kernel<T, SPW>;                                                     \
+        struct Tag {};                                                                             \
+        e = set_smem_max<Tag>(kern, ap.L.total);                                                   \
+        if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), ap.L.total, S(stream), ts, tz, ap); \
+      }
+      if (dt == CK_BF16) {
+        if (spw <= 2) CK_AWQ_STREAM(__nv_bfloat16, 2)
+        else if (spw <= 4) CK_AWQ_STREAM(__nv_bfloat16, 4)
+        else if (spw <= 6) CK_AWQ_STREAM(__nv_bfloat16, 6)
+        else CK_AWQ_STREAM(__nv_bfloat16, 8)
+      } else {
+        if (spw <= 2) CK_AWQ_STREAM(__half, 2)
+        else if (spw <= 4) CK_AWQ_STREAM(__half, 4)
+        else if (spw <= 6) CK_AWQ_STREAM(__half, 6)
+        else CK_AWQ_STREAM(__half, 8)
+      }
 #undef CK_AWQ_STREAM
-    if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_awq_w4a16: %s", cudaGetErrorString(e));
-    return launch_status("gemv_awq_w4a16");
+      if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_awq_w4a16: %s", cudaGetErrorString(e));
+      return launch_status("gemv_awq_w4a16");
+    }
   }
   const unsigned grid = (unsigned)((N + ck::awq::kRows - 1) / ck::awq::kRows);
   if (dt == CK_BF16) {

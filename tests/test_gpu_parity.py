@@ -466,6 +466,42 @@ def test_gemv_w4a8_ragged_bit_exact(ck, M, K, N, bias):
     np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
 
 
+def _tall_sample(N, seed):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.r_[0, 1, 2, N // 2, N - 2, N - 1, rng.integers(0, N, 300)])
+
+
+@pytest.mark.parametrize("M", [4, 12])
+def test_gemv_w4a8_tall_weights_bit_exact(ck, M):
+    # 2M weight rows of K = 128: each CTA's per-row scale and bias slices no
+    # longer leave room for a ring of two weight stages, so the general kernel
+    # runs; sampled output columns are checked bit for bit
+    K, N = 128, 2_000_000
+    g = torch.Generator().manual_seed(M + 77)
+    xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    xs = torch.rand(M, generator=g) * 0.1 + 0.001
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N,), 0.005, 0.02, g)
+    b = WL.uniform((N,), -1, 1, g)
+    y = ck.gemv_w4a8(xq.to(DEV), xs.to(DEV), wp.to(DEV), sw.to(DEV), b.to(DEV))
+    idx = _tall_sample(N, M)
+    r = O.gemv_w4a8(xq.numpy(), xs.numpy(), wp.numpy()[idx], to_np_f64(sw)[idx], to_np_f64(b)[idx])
+    np.testing.assert_array_equal(bf16_tensor_bits(y)[:, idx], r["y_bits"])
+
+
+def test_gemv_awq_tall_weights(ck):
+    M, K, N, G = 2, 128, 4_000_000, 64
+    g = torch.Generator().manual_seed(91)
+    x = WL.activations(M, K, 0, g)
+    qw = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    ws = WL.uniform((K // G, N), 0.001, 0.01, g)
+    wz = (torch.randn((K // G, N), generator=g) * 0.01).to(torch.bfloat16)
+    y = ck.gemv_awq_w4a16(x.to(DEV), qw.to(DEV), ws.to(DEV), wz.to(DEV), None, group_size=G)
+    idx = _tall_sample(N, 5)
+    r = O.gemv_awq_w4a16(to_np_f64(x), qw.numpy()[idx], to_np_f64(ws)[:, idx], to_np_f64(wz)[:, idx], G)
+    assert_out_close(to_np_f64(y)[:, idx], r["y_f64"])
+
+
 @pytest.mark.parametrize("M,K,N", [(5, 8192, 96), (16, 4224, 40)])
 def test_gemv_w4a8_general_path_bit_exact(ck, M, K, N):
     # K > 4096 takes the general (non-streaming) kernel
