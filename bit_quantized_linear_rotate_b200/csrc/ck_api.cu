@@ -322,11 +322,28 @@ ck_status check_input_scale(const char* who, float a, int group_size) {
   return CK_OK;
 }
 
-ck_status check_gemm_shape(const char* who, int64_t M, int64_t K, int64_t N) {
+// Largest |a * w| of one product term, per operand pair: the int32 accumulator
+// holds sum_k a * w exactly only while K * term <= INT32_MAX.
+constexpr int64_t kTermS8 = 128 * 128;      // int8 x int8
+constexpr int64_t kTermW4A8 = 128 * 8;      // int8 x (u - 8)
+constexpr int64_t kTermW4A4 = 8 * 8;        // (u - 8) x (u - 8)
+constexpr int64_t kTermLinear = 7 * 15;     // int4 code x unsigned nibble u (the linear's GEMM)
+constexpr int64_t kTermGemv = 128 * 15;     // int8 x unsigned nibble u (the W4A8 GEMV)
+
+ck_status check_acc_range(const char* who, int64_t K, int64_t term) {
+  if (K > (int64_t)INT32_MAX / term)
+    return fail(CK_ERR_UNSUPPORTED, "%s: K=%lld could overflow the int32 accumulator (K * %lld > 2^31 - 1)", who,
+                (long long)K, (long long)term);
+  return CK_OK;
+}
+
+ck_status check_gemm_shape(const char* who, int64_t M, int64_t K, int64_t N, int64_t term) {
   if (M <= 0 || K <= 0 || N <= 0) return fail(CK_ERR_INVALID_ARG, "%s: M, K, N must be > 0", who);
   if (K % 32 != 0) return fail(CK_ERR_UNSUPPORTED, "%s: K=%lld must be a multiple of 32", who, (long long)K);
   if (M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2 || K > (int64_t)INT32_MAX / 2)
     return fail(CK_ERR_UNSUPPORTED, "%s: dimension too large", who);
+  ck_status r = check_acc_range(who, K, term);
+  if (r != CK_OK) return r;
   if ((M + ck::gemm::BM - 1) / ck::gemm::BM > 65535)
     return fail(CK_ERR_UNSUPPORTED, "%s: M=%lld too large for one launch", who, (long long)M);
   return CK_OK;
@@ -586,7 +603,7 @@ ck_status ck_unpack_int4(const uint8_t* packed, int64_t R, int64_t C, int8_t* ou
 ck_status ck_gemm_s8(const int8_t* qa, const float* a_scale, int64_t M, int64_t K, int64_t N,
                      const int8_t* w, const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
                      void* stream) {
-  ck_status r = check_gemm_shape("gemm_s8", M, K, N);
+  ck_status r = check_gemm_shape("gemm_s8", M, K, N, kTermS8);
   if (r != CK_OK) return r;
   if (!qa || !a_scale || !w || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemm_s8: null pointer");
   if (!aligned(qa, 16) || !aligned(w, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_s8: operands must be 16-byte aligned");
@@ -598,7 +615,7 @@ ck_status ck_gemm_s8(const int8_t* qa, const float* a_scale, int64_t M, int64_t 
 ck_status ck_gemm_w4a8(const int8_t* qa, const float* a_scale, int64_t M, int64_t K, int64_t N,
                        const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
                        uint16_t* y, void* stream) {
-  ck_status r = check_gemm_shape("gemm_w4a8", M, K, N);
+  ck_status r = check_gemm_shape("gemm_w4a8", M, K, N, kTermW4A8);
   if (r != CK_OK) return r;
   if (!qa || !a_scale || !w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8: null pointer");
   if (!aligned(qa, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a8: operands must be 16-byte aligned");
@@ -609,7 +626,7 @@ ck_status ck_gemm_w4a8(const int8_t* qa, const float* a_scale, int64_t M, int64_
 
 ck_status ck_gemm_s8_i32(const int8_t* qa, const int8_t* w, int64_t M, int64_t K, int64_t N, int32_t* acc,
                          void* stream) {
-  ck_status r = check_gemm_shape("gemm_s8_i32", M, K, N);
+  ck_status r = check_gemm_shape("gemm_s8_i32", M, K, N, kTermS8);
   if (r != CK_OK) return r;
   if (!qa || !w || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_s8_i32: null pointer");
   if (!aligned(qa, 16) || !aligned(w, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_s8_i32: operands must be 16-byte aligned");
@@ -620,7 +637,7 @@ ck_status ck_gemm_s8_i32(const int8_t* qa, const int8_t* w, int64_t M, int64_t K
 ck_status ck_gemm_w4a4(const uint8_t* qa_packed, const float* a_scale, int64_t M, int64_t K,
                        int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
                        const uint16_t* bias, uint16_t* y, void* stream) {
-  ck_status r = check_gemm_shape("gemm_w4a4", M, K, N);
+  ck_status r = check_gemm_shape("gemm_w4a4", M, K, N, kTermW4A4);
   if (r != CK_OK) return r;
   if (!qa_packed || !a_scale || !w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4: null pointer");
   if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4: operands must be 16-byte aligned");
@@ -640,7 +657,7 @@ namespace {
 
 ck_status linear_quantize_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
                                 int group_size, float in_scale, void* workspace, size_t ws_bytes, void* stream) {
-  ck_status r = check_gemm_shape(who, M, K, 1);
+  ck_status r = check_gemm_shape(who, M, K, 1, kTermLinear);
   if (r != CK_OK) return r;
   if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
   if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "%s: unknown dtype", who);
@@ -670,7 +687,7 @@ ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t
 ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
                                 const uint16_t* bias, uint16_t* y, const void* workspace, size_t ws_bytes,
                                 void* stream) {
-  ck_status r = check_gemm_shape("linear_w4a4_matmul", M, K, N);
+  ck_status r = check_gemm_shape("linear_w4a4_matmul", M, K, N, kTermLinear);
   if (r != CK_OK) return r;
   if ((r = check_linear_workspace("linear_w4a4_matmul", M, K, workspace, ws_bytes)) != CK_OK) return r;
   if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_matmul: null pointer");
@@ -697,7 +714,7 @@ namespace {
 ck_status linear_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
                        int group_size, float in_scale, const uint8_t* w_packed, const uint16_t* w_scale,
                        const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
-  ck_status r = check_gemm_shape(who, M, K, N);
+  ck_status r = check_gemm_shape(who, M, K, N, kTermLinear);
   if (r != CK_OK) return r;
   // validate both phases before enqueuing either
   if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
@@ -775,7 +792,7 @@ ck_status ck_linear_w4a4_static(const void* x, ck_dtype xt, int64_t M, int64_t K
                                 int64_t ldx, int group_size, const uint8_t* w_packed,
                                 const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
                                 void* stream) {
-  ck_status r = check_gemm_shape("linear_w4a4_static", M, K, N);
+  ck_status r = check_gemm_shape("linear_w4a4_static", M, K, N, kTermLinear);
   if (r != CK_OK) return r;
   const size_t need = linear_ws_bytes(M, K);
   if (need > (size_t)CK_LINEAR_STATIC_SCRATCH_BYTES)
@@ -791,7 +808,7 @@ ck_status ck_linear_w4a4_static(const void* x, ck_dtype xt, int64_t M, int64_t K
 
 ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, int64_t M, int64_t K,
                            int64_t N, int32_t* acc, void* stream) {
-  ck_status r = check_gemm_shape("gemm_w4a4_i32", M, K, N);
+  ck_status r = check_gemm_shape("gemm_w4a4_i32", M, K, N, kTermW4A4);
   if (r != CK_OK) return r;
   if (!qa_packed || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a4_i32: null pointer");
   if (!aligned(qa_packed, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a4_i32: operands must be 16-byte aligned");
@@ -801,7 +818,7 @@ ck_status ck_gemm_w4a4_i32(const uint8_t* qa_packed, const uint8_t* w_packed, in
 
 ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M, int64_t K, int64_t N,
                            int32_t* acc, void* stream) {
-  ck_status r = check_gemm_shape("gemm_w4a8_i32", M, K, N);
+  ck_status r = check_gemm_shape("gemm_w4a8_i32", M, K, N, kTermW4A8);
   if (r != CK_OK) return r;
   if (!qa || !w_packed || !acc) return fail(CK_ERR_INVALID_ARG, "gemm_w4a8_i32: null pointer");
   if (!aligned(qa, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemm_w4a8_i32: operands must be 16-byte aligned");
@@ -816,6 +833,7 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
   if (M > 16) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: M=%lld > 16", (long long)M);
   if (K % 128 != 0) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: K must be a multiple of 128");
   if (K > INT32_MAX / 2 || N > INT32_MAX / 2) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: dimension too large");
+  if (check_acc_range("gemv_w4a8", K, kTermGemv) != CK_OK) return CK_ERR_UNSUPPORTED;
   if (!xq || !x_scale || !w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemv_w4a8: null pointer");
   if (!aligned(xq, 16) || !aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8: operands must be 16-byte aligned");
   if (!aligned(x_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))

@@ -20,6 +20,11 @@
  *   the kernels decline (the pages' "unsupported-shape decline"); CK_ERR_CUDA
  *   when a launch fails. Nothing is enqueued when validation fails.
  *   ck_last_error() returns a thread-local message for the last failure.
+ * - Integer accumulation is exact int32. A shape whose K could overflow it is
+ *   CK_ERR_UNSUPPORTED: K must satisfy K * max|a * w| <= 2^31 - 1. The
+ *   largest term is 128 * 128 for int8 x int8 (K <= 131071), 128 * 8 for
+ *   int8 x int4 (K <= 2097151), 8 * 8 for int4 x int4, 7 * 15 in the linear,
+ *   and 128 * 15 in the W4A8 GEMV (K <= 1118481).
  * - Kernels that wait on shared-memory barriers give up after a bounded time
  *   and set a device error word instead of hanging; ck_device_error_check()
  *   reports it.

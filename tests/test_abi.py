@@ -179,6 +179,23 @@ def test_input_scale_other_checks(ck):
     assert lin(64, 1.0, ws - 1) == ck.CK_ERR_INVALID_ARG
 
 
+def test_k_that_could_overflow_the_int32_accumulator_is_rejected(ck):
+    # |sum_k a w| <= K * max|a w|: int8 x int8 128 * 128, int8 x int4 128 * 8,
+    # int4 x int4 8 * 8, int8 x unsigned nibble (GEMV) 128 * 15
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    g = (P(1 << 20), P(1 << 20), 8)
+    tail = (P(1 << 20), P(1 << 20), None, P(1 << 20), None)
+    assert L.ck_gemm_s8(*g[:2], 8, 131072, 8, *tail) == ck.CK_ERR_UNSUPPORTED
+    assert "overflow" in ck.last_error()
+    assert L.ck_gemm_s8_i32(P(1 << 20), P(1 << 20), 8, 131072, 8, P(1 << 20), None) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemm_w4a8(*g[:2], 8, 2097152, 8, *tail) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemm_w4a4(*g[:2], 8, 33554432, 8, *tail) == ck.CK_ERR_UNSUPPORTED
+    assert L.ck_gemv_w4a8(P(1 << 20), P(1 << 20), 4, 1118592, 8, P(1 << 20), P(1 << 20), None, P(1 << 20),
+                          None) == ck.CK_ERR_UNSUPPORTED
+    assert "overflow" in ck.last_error()
+
+
 def test_selftest_timeout_range_is_validated(ck):
     assert ck.lib.ck_selftest_bounded_wait(10, None) == ck.CK_ERR_INVALID_ARG
     assert ck.lib.ck_selftest_bounded_wait(10 ** 10, None) == ck.CK_ERR_INVALID_ARG
