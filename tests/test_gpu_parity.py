@@ -609,6 +609,63 @@ def test_back_to_back_linear_calls_share_a_workspace(ck):
     ck.device_error_check()
 
 
+def test_graph_replay_equals_eager_calls(ck):
+    """Chains of calls captured once in a CUDA graph and replayed (how the bench times the GEMVs
+    and the other configs): every output equals the eager call's, bit for bit."""
+    g = torch.Generator().manual_seed(123)
+    K8, N8 = 4096, 2048
+    wps = [torch.randint(0, 256, (N8, K8 // 2), generator=g, dtype=torch.uint8).to(DEV) for _ in range(3)]
+    sw = WL.uniform((N8,), 0.005, 0.02, g).to(DEV)
+    xqs = {M: torch.randint(-127, 128, (M, K8), generator=g, dtype=torch.int8).to(DEV) for M in (4, 16)}
+    xss = {M: (torch.rand(M, generator=g) * 0.1 + 0.001).to(DEV) for M in (4, 16)}
+    Ka, Na, G = 3072, 2048, 64
+    xa = WL.activations(2, Ka, 0, g).to(DEV)
+    qws = [torch.randint(0, 256, (Na, Ka // 2), generator=g, dtype=torch.uint8).to(DEV) for _ in range(3)]
+    wsa = WL.uniform((Ka // G, Na), 0.001, 0.01, g).to(DEV)
+    wza = (torch.randn((Ka // G, Na), generator=g) * 0.01).to(torch.bfloat16).to(DEV)
+    lin = {M: WL.small_linear_inputs(M, 1024, 520, seed=M, n_outlier_cols=10, with_bias=True) for M in (300, 32)}
+    lin = {M: {k: v.to(DEV) for k, v in d.items()} for M, d in lin.items()}
+    wss = {M: torch.empty(ck.linear_w4a4_workspace_bytes(M, 1024), device=DEV, dtype=torch.uint8) for M in lin}
+    xr = WL.activations(257, 3840, 38, g).to(DEV)
+
+    def chain(outs):
+        i = 0
+        for c in range(3):
+            for M in (4, 16):
+                ck.gemv_w4a8(xqs[M], xss[M], wps[c], sw, out=outs[i]); i += 1
+            ck.gemv_awq_w4a16(xa, qws[c], wsa, wza, group_size=G, out=outs[i]); i += 1
+        for M, d in lin.items():
+            ck.linear_w4a4(d["x"], d["w_packed"], d["w_scale"], G, bias=d["bias"], workspace=wss[M], out=outs[i])
+            i += 1
+        ck.rotate_quant_rowwise(xr, 64, 4, q_out=outs[i], scale_out=outs[i + 1])
+
+    def make_outs():
+        o = []
+        for c in range(3):
+            o += [torch.empty(M, N8, device=DEV, dtype=torch.bfloat16) for M in (4, 16)]
+            o.append(torch.empty(2, Na, device=DEV, dtype=torch.bfloat16))
+        o += [torch.empty(M, 520, device=DEV, dtype=torch.bfloat16) for M in lin]
+        o += [torch.empty(257, 1920, device=DEV, dtype=torch.uint8), torch.empty(257, device=DEV)]
+        return o
+
+    ref = make_outs()
+    chain(ref)                 # eager; also fills the library's per-kernel caches before capture
+    torch.cuda.synchronize()
+    got = make_outs()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        chain(got)
+    for _ in range(3):
+        for t in got:
+            t.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        for a, b in zip(got, ref):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    del graph
+    ck.device_error_check()
+
+
 def test_back_to_back_dependent_gemvs(ck):
     """A chain of GEMVs where each call reads the previous call's output, launched back to back:
     every activation read must see the previous kernel's writes."""
