@@ -38,6 +38,30 @@ def test_library_exports_every_declared_symbol(ck):
         assert name in ck.SIGNATURES, f"binding lacks {name}"
 
 
+def test_header_is_plain_c_and_links_from_c(ck, tmp_path):
+    # the boundary is a C ABI: ck.h compiles as strict C99 and a C program links
+    # against libck.so and calls it (M = 0 is a no-op that needs no GPU)
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_ck.c"
+    src.write_text('#include "ck.h"\n#include <stdio.h>\n'
+                   "int main(void) {\n"
+                   '  printf("%s\\n", ck_version());\n'
+                   "  return ck_rotate_quant_rowwise(0, CK_BF16, 0, 64, 64, 64, 4, 0, 0, 0) == CK_OK ? 0 : 1;\n"
+                   "}\n")
+    libdir = os.path.dirname(ck.LIB_PATH)
+    exe = tmp_path / "use_ck"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-l:libck.so", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0
+    assert "sm_100a" in out.stdout
+
+
 def test_version_and_last_error(ck):
     assert "sm_100a" in ck.version()
     assert isinstance(ck.last_error(), str)
