@@ -53,6 +53,7 @@ SIGNATURES = {
                               _p],
     "ck_linear_w4a4_static": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "ck_gemv_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+    "ck_gemv_w4a8_tc": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemv_awq_w4a16": [_p, _int, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p],
     "ck_gemm_w4a4_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
     "ck_gemm_w4a8_i32": [_p, _p, _i64, _i64, _i64, _p, _p],
@@ -343,6 +344,18 @@ def gemv_w4a8(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
         out = torch.empty((M, N), device=xq.device, dtype=torch.bfloat16)
     _check(lib.ck_gemv_w4a8(_ptr(xq), _ptr(x_scale), M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias),
                             _ptr(out), _stream(stream)), "ck_gemv_w4a8")
+    return out
+
+
+def gemv_w4a8_tc(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
+    """gemv_w4a8 on the tcgen05 tensor cores (the same results bit for bit; an alternative path)."""
+    _cuda(xq, x_scale, w_packed, w_scale, bias)
+    M, K = xq.shape
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), device=xq.device, dtype=torch.bfloat16)
+    _check(lib.ck_gemv_w4a8_tc(_ptr(xq), _ptr(x_scale), M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias),
+                               _ptr(out), _stream(stream)), "ck_gemv_w4a8_tc")
     return out
 
 

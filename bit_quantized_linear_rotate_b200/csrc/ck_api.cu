@@ -21,6 +21,7 @@
 #include "gemv_awq.cuh"
 #include "gemv_stream.cuh"
 #include "gemv_w4a8.cuh"
+#include "gemv_w4a8_tc.cuh"
 #include "rotate_quant.cuh"
 #include "rotate_quant_general.cuh"
 
@@ -826,6 +827,63 @@ ck_status ck_gemm_w4a8_i32(const int8_t* qa, const uint8_t* w_packed, int64_t M,
   return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_PACKED4, ck::gemm::EPI_I32>(qa, M, K, N, w_packed, nullptr, nullptr, nullptr, nullptr, acc, S(stream));
 }
 
+}  // extern "C"
+
+namespace {
+
+// W4A8 GEMV on the tensor cores: ceil(N / 128) row blocks, each one cluster of
+// `split` CTAs dividing K. One wave at one CTA per SM sets the split (at most 8
+// and at most K / 128), raised where a CTA's activations would not fit.
+ck_status gemv_w4a8_tc_launch(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
+                              const uint8_t* w_packed, const __nv_bfloat16* sw, const __nv_bfloat16* bb,
+                              __nv_bfloat16* yy, cudaStream_t st) {
+  using namespace ck::gtc;
+  constexpr int kSmemMax = 227 * 1024;
+  const int nkb = (int)(K / BK);
+  const int64_t rb = (N + BM - 1) / BM;
+  const int split_max = std::min(8, nkb);
+  int split = (int)std::max<int64_t>(1, std::min<int64_t>(split_max, sm_count() / rb));
+  while (split < split_max && smem_bytes((nkb + split - 1) / split) > kSmemMax) ++split;
+  const int nkbc_max = (nkb + split - 1) / split;
+  const int smem = smem_bytes(nkbc_max);
+  if (smem > kSmemMax) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8_tc: K=%lld too large", (long long)K);
+  if (rb * split > INT32_MAX) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8_tc: N=%lld too large", (long long)N);
+  CUtensorMap tw, tx;
+  ck_status r = make_tmap(&tw, w_packed, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, PKB, BM,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (r != CK_OK) return r;
+  r = make_tmap(&tx, xq, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (r != CK_OK) return r;
+  auto kern = gemv_w4a8_tc_kernel;
+  struct Tag {};
+  if ((r = ensure_smem_attr<Tag>(kern, kSmemMax)) != CK_OK) return r;
+  Params p;
+  p.M = (int)M; p.K = (int)K; p.N = (int)N;
+  p.S = split; p.nkb = nkb; p.nkbc_max = nkbc_max;
+  p.xs = x_scale; p.sw = sw; p.bias = bb; p.y = yy;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((unsigned)(rb * split), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
+  if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8_tc: launch failed: %s", cudaGetErrorString(e));
+  return launch_status("gemv_w4a8_tc");
+}
+
+}  // namespace
+
+extern "C" {
+
 ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
                        const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
                        uint16_t* y, void* stream) {
@@ -909,6 +967,24 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
   else
     ck::w4a8::gemv_w4a8_kernel<2><<<grid, ck::w4a8::kWarps * 32, 0, S(stream)>>>(xq, x_scale, (int)M, (int)K, (int)N, w_packed, sw, bb, yy);
   return launch_status("gemv_w4a8");
+}
+
+ck_status ck_gemv_w4a8_tc(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
+                          const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
+                          uint16_t* y, void* stream) {
+  if (M <= 0 || K <= 0 || N <= 0) return fail(CK_ERR_INVALID_ARG, "gemv_w4a8_tc: M, K, N must be > 0");
+  if (M > 16) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8_tc: M=%lld > 16", (long long)M);
+  if (K % 128 != 0) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8_tc: K must be a multiple of 128");
+  if (K > 8192) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8_tc: K=%lld > 8192", (long long)K);
+  if (N > INT32_MAX / 2) return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8_tc: dimension too large");
+  if (!xq || !x_scale || !w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "gemv_w4a8_tc: null pointer");
+  if (!aligned(xq, 16) || !aligned(w_packed, 16))
+    return fail(CK_ERR_UNSUPPORTED, "gemv_w4a8_tc: operands must be 16-byte aligned");
+  if (!aligned(x_scale, 4) || !aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "gemv_w4a8_tc: misaligned scale, bias or output");
+  return gemv_w4a8_tc_launch(xq, x_scale, M, K, N, w_packed, reinterpret_cast<const __nv_bfloat16*>(w_scale),
+                             reinterpret_cast<const __nv_bfloat16*>(bias), reinterpret_cast<__nv_bfloat16*>(y),
+                             S(stream));
 }
 
 ck_status ck_gemv_awq_w4a16(const void* x, ck_dtype dt, int64_t M, int64_t K, int64_t N, int group_size,

@@ -288,6 +288,20 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
                        uint16_t* y, void* stream);
 
 /*
+ * ck_gemv_w4a8 computed on the tcgen05 tensor cores: 128 weight rows are the
+ * MMA's M operand (decoded to unsigned bytes in shared memory), the activation
+ * rows padded to 16 its N operand, and clusters of CTAs split K where the
+ * row blocks are too few. The results equal ck_gemv_w4a8's bit for bit. It
+ * is an alternative path, not the default: on K = 4096, N = 12288 it is
+ * currently about twice as slow as ck_gemv_w4a8, whose legacy-MMA streaming
+ * kernels ck_gemv_w4a8 keeps using.
+ * Arguments and errors as for ck_gemv_w4a8, with K <= 8192.
+ */
+ck_status ck_gemv_w4a8_tc(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
+                          const uint8_t* w_packed, const uint16_t* w_scale, const uint16_t* bias,
+                          uint16_t* y, void* stream);
+
+/*
  * AWQ W4A16 GEMV ("ck.gemv_awq_w4a16(x, qdata, wscales, wzeros, bias=,
  * group_size=)", comfy_kitchen/tensor/awq_w4a16.py, _awq_forward):
  *   W[n,k] = (u[n,k] - 8) * wscales[k/G, n] + wzeros[k/G, n]

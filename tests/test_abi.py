@@ -150,6 +150,19 @@ def test_gemv_validation(ck):
     assert L.ck_gemv_awq_w4a16(P(1 << 20), 5, 2, 128, 8, 64, P(1 << 20), P(1 << 20), P(1 << 20), None, P(1 << 20), None) == ck.CK_ERR_INVALID_ARG
 
 
+def test_tensor_core_gemv_validation(ck):
+    P = lambda v: ctypes.c_void_p(v)
+    L = ck.lib
+    call = lambda M, K, N, xq=P(1 << 20): L.ck_gemv_w4a8_tc(xq, P(1 << 20), M, K, N, P(1 << 20), P(1 << 20), None,
+                                                               P(1 << 20), None)
+    assert call(17, 128, 8) == ck.CK_ERR_UNSUPPORTED        # M > 16
+    assert call(4, 96, 8) == ck.CK_ERR_UNSUPPORTED          # K % 128
+    assert call(4, 8320, 8) == ck.CK_ERR_UNSUPPORTED        # K > 8192
+    assert call(0, 128, 8) == ck.CK_ERR_INVALID_ARG
+    assert call(4, 128, 8, xq=None) == ck.CK_ERR_INVALID_ARG
+    assert call(4, 128, 8, xq=P((1 << 20) + 8)) == ck.CK_ERR_UNSUPPORTED
+
+
 def test_general_rotation_validation(ck):
     P = lambda v: ctypes.c_void_p(v)
     L = ck.lib

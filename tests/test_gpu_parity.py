@@ -515,6 +515,35 @@ def test_gemv_w4a8_general_path_bit_exact(ck, M, K, N):
     np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
 
 
+@pytest.mark.parametrize("M,K,N,bias", [(3, 256, 100, True), (1, 128, 300, False), (9, 512, 37, True),
+                                         (16, 1280, 48, True), (5, 8192, 96, False), (12, 4096, 1000, True),
+                                         (16, 3840, 3840, False)])
+def test_gemv_w4a8_tc_bit_exact(ck, M, K, N, bias):
+    # the tensor-core GEMV against the oracle and the default GEMV, bit for bit
+    g = torch.Generator().manual_seed(M * K + N)
+    xq = torch.randint(-128, 128, (M, K), generator=g, dtype=torch.int8)
+    xs = torch.rand(M, generator=g) * 0.1 + 0.001
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N,), 0.005, 0.02, g)
+    b = WL.uniform((N,), -1, 1, g) if bias else None
+    args = (xq.to(DEV), xs.to(DEV), wp.to(DEV), sw.to(DEV), None if b is None else b.to(DEV))
+    y = ck.gemv_w4a8_tc(*args)
+    r = O.gemv_w4a8(xq.numpy(), xs.numpy(), wp.numpy(), to_np_f64(sw), None if b is None else to_np_f64(b))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
+    assert np.array_equal(bf16_tensor_bits(ck.gemv_w4a8(*args)), bf16_tensor_bits(y))
+
+
+@pytest.mark.parametrize("M", WL.GEMV_W4A8.Ms)
+def test_gemv_w4a8_tc_config_equals_default(ck, M):
+    d = WL.gemv_w4a8_inputs(WL.GEMV_W4A8, M)
+    xq, xs = ck.rotate_quant_rowwise(d["x"].to(DEV), 1, 8)
+    wp, sw = d["w_packed"].to(DEV), d["w_scale"].to(DEV)
+    y_tc = ck.gemv_w4a8_tc(xq, xs, wp, sw)
+    y = ck.gemv_w4a8(xq, xs, wp, sw)
+    torch.cuda.synchronize()
+    assert torch.equal(y_tc.view(torch.int16), y.view(torch.int16))
+
+
 def test_gemv_w4a8_agrees_with_large_m_gemm(ck):
     # the decode GEMV and the tensor-core GEMM share codec and epilogue: same int32 results
     g = torch.Generator().manual_seed(5)
