@@ -12,6 +12,7 @@ Cases (full workload sizes, a few GB at most on the device):
   linmm_M8192      ck_linear_w4a4_matmul (the linear's GEMM phase alone)
   linq_M8192       ck_linear_w4a4_quantize (the linear's rotate + quantize phase alone)
   w4a8_M{1,4,16}   ck_gemv_w4a8, K=4096, N=12288
+  w4a8tc_M{1,4,16} ck_gemv_w4a8_tc (the tcgen05 alternative), same shapes
   awq_M{1,2,4}     ck_gemv_awq_w4a16, K=3072, N=18432, G=64
 One warm-up call precedes the timed iterations; the process exits non-zero if
 a kernel reported an error.
@@ -56,12 +57,15 @@ def build_case(name: str, dev):
         if name == "linmm_M8192":
             ck.linear_w4a4_quantize(x, w.G, ws)
             return lambda: ck.linear_w4a4_matmul(w.M, w.K, wp, sw, ws, out=y)
-    if name.startswith("w4a8_M"):
-        M = int(name[len("w4a8_M"):])
+    if name.startswith(("w4a8_M", "w4a8tc_M")):
+        tc = name.startswith("w4a8tc_M")
+        M = int(name[len("w4a8tc_M" if tc else "w4a8_M"):])
         d = WL.gemv_w4a8_inputs(WL.GEMV_W4A8, M)
         xq, xs = ck.rotate_quant_rowwise(d["x"].to(dev), 1, 8)
         wp, sw = d["w_packed"].to(dev), d["w_scale"].to(dev)
         y = torch.empty(M, WL.GEMV_W4A8.N, device=dev, dtype=torch.bfloat16)
+        if tc:
+            return lambda: ck.gemv_w4a8_tc(xq, xs, wp, sw, out=y)
         return lambda: ck.gemv_w4a8(xq, xs, wp, sw, out=y)
     if name.startswith("awq_M"):
         M = int(name[len("awq_M"):])
