@@ -101,6 +101,24 @@ def _dtype_code(dt) -> int:
     raise TypeError(f"unsupported dtype {dt} (bf16 or fp16)")
 
 
+_BYTES = (torch.uint8, torch.int8)      # codes and packed nibbles: either view of the same bytes
+_HALF = (torch.bfloat16, torch.float16)
+_F32 = (torch.float32,)
+_BF16 = (torch.bfloat16,)
+_I32 = (torch.int32,)
+
+
+def _types(where: str, **named) -> None:
+    """TypeError unless each named tensor (None is skipped) has one of its allowed dtypes.
+
+    The C entry points see raw bytes, so a tensor of the wrong dtype would be
+    read as garbage rather than rejected."""
+    for name, (t, allowed) in named.items():
+        if t is not None and t.dtype not in allowed:
+            want = " or ".join(str(a).replace("torch.", "") for a in allowed)
+            raise TypeError(f"{where}: {name} must be {want}, got {str(t.dtype).replace('torch.', '')}")
+
+
 def _cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
@@ -128,6 +146,7 @@ def last_error() -> str:
 
 def rotate_quant_rowwise(x, group_size: int, bits: int, q_out=None, scale_out=None, stream=None):
     """Returns (q, scale): q packed int4 (..., K/2) uint8 for bits=4, int8 (..., K) for bits=8."""
+    _types("rotate_quant_rowwise", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
     _cuda(x)
     M, K, ldx, x2 = _rows(x)
     lead = tuple(x.shape[:-1])
@@ -145,6 +164,7 @@ def rotate_quant_rowwise(x, group_size: int, bits: int, q_out=None, scale_out=No
 
 def rotate_quant_rowwise_i8(x, group_size: int, bits: int, q_out=None, scale_out=None, stream=None):
     """Returns (q, scale) with the codes stored one per byte: q (..., K) int8 for bits 4 or 8."""
+    _types("rotate_quant_rowwise_i8", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
     _cuda(x)
     M, K, ldx, x2 = _rows(x)
     lead = tuple(x.shape[:-1])
@@ -165,6 +185,7 @@ def rotate_quant_rowwise_r(x, R, bits: int, q_out=None, scale_out=None, stream=N
     Returns (q, s) in the formats of rotate_quant_rowwise: bits=4 packed (..., K/2) uint8, bits=8
     (..., K) int8; s (...) float32.
     """
+    _types("rotate_quant_rowwise_r", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
     _cuda(x, R)
     if R.dtype != torch.float32 or R.dim() != 2 or R.shape[0] != R.shape[1] or not R.is_contiguous():
         raise ValueError("R must be a contiguous square float32 matrix")
@@ -184,6 +205,7 @@ def rotate_quant_rowwise_r(x, R, bits: int, q_out=None, scale_out=None, stream=N
 def rotate_quant_rowwise_scaled(x, group_size: int, bits: int, input_scale: float, q_out=None,
                                 scale_out=None, stream=None):
     """rotate_quant_rowwise of input_scale * x (a finite tensor-wise scale >= 0); same formats."""
+    _types("rotate_quant_rowwise_scaled", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
     _cuda(x)
     M, K, ldx, x2 = _rows(x)
     lead = tuple(x.shape[:-1])
@@ -201,6 +223,7 @@ def rotate_quant_rowwise_scaled(x, group_size: int, bits: int, input_scale: floa
 
 def unpack_int4(packed, out=None, stream=None):
     """(R, C/2) packed int4 -> (R, C) int8 with value u - 8."""
+    _types("unpack_int4", packed=(packed, _BYTES), out=(out, _BYTES))
     _cuda(packed)
     R, Ch = packed.shape
     if out is None:
@@ -211,6 +234,8 @@ def unpack_int4(packed, out=None, stream=None):
 
 def gemm_w4a8(qa, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):
     """int8 activation codes (M, K) x packed int4 weights (N, K/2) -> bf16 (M, N)."""
+    _types("gemm_w4a8", qa=(qa, _BYTES), a_scale=(a_scale, _F32), w_packed=(w_packed, _BYTES),
+           w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
     _cuda(qa, a_scale, w_packed, w_scale, bias)
     M, K = qa.shape
     N = w_packed.shape[0]
@@ -222,6 +247,8 @@ def gemm_w4a8(qa, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):
 
 
 def gemm_s8(qa, a_scale, w8, w_scale, bias=None, out=None, stream=None):
+    _types("gemm_s8", qa=(qa, _BYTES), a_scale=(a_scale, _F32), w8=(w8, _BYTES), w_scale=(w_scale, _BF16),
+           bias=(bias, _BF16), out=(out, _BF16))
     _cuda(qa, a_scale, w8, w_scale, bias)
     M, K = qa.shape
     N = w8.shape[0]
@@ -233,6 +260,7 @@ def gemm_s8(qa, a_scale, w8, w_scale, bias=None, out=None, stream=None):
 
 
 def gemm_s8_i32(qa, w8, out=None, stream=None):
+    _types("gemm_s8_i32", qa=(qa, _BYTES), w8=(w8, _BYTES), out=(out, _I32))
     _cuda(qa, w8)
     M, K = qa.shape
     N = w8.shape[0]
@@ -243,6 +271,8 @@ def gemm_s8_i32(qa, w8, out=None, stream=None):
 
 
 def gemm_w4a4(qa_packed, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):
+    _types("gemm_w4a4", qa_packed=(qa_packed, _BYTES), a_scale=(a_scale, _F32), w_packed=(w_packed, _BYTES),
+           w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
     _cuda(qa_packed, a_scale, w_packed, w_scale, bias)
     M, Kh = qa_packed.shape
     N = w_packed.shape[0]
@@ -260,6 +290,8 @@ def linear_w4a4_workspace_bytes(M: int, K: int) -> int:
 def linear_w4a4(x, w_packed, w_scale, group_size: int, bias=None, workspace=None, out=None,
                 stream=None):
     """ConvRot W4A4 linear: y (..., N) bf16 from x (..., K) bf16/fp16 and packed (N, K/2) weights."""
+    _types("linear_w4a4", x=(x, _HALF), w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
+           out=(out, _BF16))
     _cuda(x, w_packed, w_scale, bias)
     M, K, ldx, x2 = _rows(x)
     N = w_packed.shape[0]
@@ -278,6 +310,8 @@ def linear_w4a4(x, w_packed, w_scale, group_size: int, bias=None, workspace=None
 def linear_w4a4_scaled(x, w_packed, w_scale, group_size: int, input_scale: float, bias=None, workspace=None,
                        out=None, stream=None):
     """linear_w4a4 of input_scale * x (a finite tensor-wise scale >= 0); the output is not rescaled."""
+    _types("linear_w4a4_scaled", x=(x, _HALF), w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
+           out=(out, _BF16))
     _cuda(x, w_packed, w_scale, bias)
     M, K, ldx, x2 = _rows(x)
     N = w_packed.shape[0]
@@ -303,6 +337,8 @@ def linear_w4a4_static(x, w_packed, w_scale, group_size: int, bias=None, out=Non
     Same results as linear_w4a4. Calls on one device share that scratch, so calls that may run
     at the same time on the GPU (different streams, several threads) must not be mixed.
     """
+    _types("linear_w4a4_static", x=(x, _HALF), w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
+           out=(out, _BF16))
     _cuda(x, w_packed, w_scale, bias)
     M, K, ldx, x2 = _rows(x)
     N = w_packed.shape[0]
@@ -316,6 +352,7 @@ def linear_w4a4_static(x, w_packed, w_scale, group_size: int, bias=None, out=Non
 
 def linear_w4a4_quantize(x, group_size: int, workspace, stream=None):
     """Phase 1 of linear_w4a4: rotate + quantize x into `workspace` (opaque)."""
+    _types("linear_w4a4_quantize", x=(x, _HALF))
     _cuda(x, workspace)
     M, K, ldx, x2 = _rows(x)
     _check(lib.ck_linear_w4a4_quantize(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, _ptr(workspace),
@@ -326,6 +363,8 @@ def linear_w4a4_quantize(x, group_size: int, workspace, stream=None):
 
 def linear_w4a4_matmul(M: int, K: int, w_packed, w_scale, workspace, bias=None, out=None, stream=None):
     """Phase 2 of linear_w4a4: GEMM of the workspace codes with the packed weights -> y (M, N) bf16."""
+    _types("linear_w4a4_matmul", w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
+           out=(out, _BF16))
     _cuda(w_packed, w_scale, workspace, bias)
     N = w_packed.shape[0]
     if out is None:
@@ -337,6 +376,8 @@ def linear_w4a4_matmul(M: int, K: int, w_packed, w_scale, workspace, bias=None, 
 
 
 def gemv_w4a8(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
+    _types("gemv_w4a8", xq=(xq, _BYTES), x_scale=(x_scale, _F32), w_packed=(w_packed, _BYTES),
+           w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
     _cuda(xq, x_scale, w_packed, w_scale, bias)
     M, K = xq.shape
     N = w_packed.shape[0]
@@ -349,6 +390,8 @@ def gemv_w4a8(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
 
 def gemv_w4a8_tc(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
     """gemv_w4a8 on the tcgen05 tensor cores (the same results bit for bit; an alternative path)."""
+    _types("gemv_w4a8_tc", xq=(xq, _BYTES), x_scale=(x_scale, _F32), w_packed=(w_packed, _BYTES),
+           w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
     _cuda(xq, x_scale, w_packed, w_scale, bias)
     M, K = xq.shape
     N = w_packed.shape[0]
@@ -361,6 +404,9 @@ def gemv_w4a8_tc(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=Non
 
 def gemv_awq_w4a16(x, qweight, wscales, wzeros, bias=None, group_size: int = 64, out=None, stream=None):
     """``ck.gemv_awq_w4a16(x, qdata, wscales, wzeros, bias=, group_size=)``."""
+    same = (x.dtype,) if x.dtype in _HALF else _HALF
+    _types("gemv_awq_w4a16", x=(x, _HALF), qweight=(qweight, _BYTES), wscales=(wscales, same),
+           wzeros=(wzeros, same), bias=(bias, same), out=(out, same))
     _cuda(x, qweight, wscales, wzeros, bias)
     M, K = x.shape
     N = qweight.shape[0]
@@ -373,6 +419,7 @@ def gemv_awq_w4a16(x, qweight, wscales, wzeros, bias=None, group_size: int = 64,
 
 
 def gemm_w4a4_i32(qa_packed, w_packed, out=None, stream=None):
+    _types("gemm_w4a4_i32", qa_packed=(qa_packed, _BYTES), w_packed=(w_packed, _BYTES), out=(out, _I32))
     _cuda(qa_packed, w_packed)
     M, Kh = qa_packed.shape
     N = w_packed.shape[0]
@@ -384,6 +431,7 @@ def gemm_w4a4_i32(qa_packed, w_packed, out=None, stream=None):
 
 
 def gemm_w4a8_i32(qa, w_packed, out=None, stream=None):
+    _types("gemm_w4a8_i32", qa=(qa, _BYTES), w_packed=(w_packed, _BYTES), out=(out, _I32))
     _cuda(qa, w_packed)
     M, K = qa.shape
     N = w_packed.shape[0]

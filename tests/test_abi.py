@@ -246,3 +246,36 @@ def test_package_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def test_binding_rejects_wrong_dtypes_before_any_launch(ck):
+    # the C entry points see bytes: the binding checks dtypes first (CPU tensors
+    # with the right dtypes then fail the CUDA-tensor check, so no launch happens)
+    import torch
+    i8 = torch.zeros(4, 128, dtype=torch.int8)
+    u8 = torch.zeros(8, 64, dtype=torch.uint8)
+    f32 = torch.ones(4)
+    bf = torch.ones(8, dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="x_scale"):
+        ck.gemv_w4a8(i8, f32.to(torch.bfloat16), u8, bf)
+    with pytest.raises(TypeError, match="w_scale"):
+        ck.gemv_w4a8(i8, f32, u8, bf.float())
+    with pytest.raises(TypeError, match="xq"):
+        ck.gemv_w4a8_tc(i8.float(), f32, u8, bf)
+    with pytest.raises(ValueError, match="CUDA"):
+        ck.gemv_w4a8(i8, f32, u8, bf)
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="x"):
+        ck.rotate_quant_rowwise(x.float(), 64, 4)
+    with pytest.raises(TypeError, match="scale_out"):
+        ck.rotate_quant_rowwise(x, 64, 4, scale_out=torch.empty(4, dtype=torch.float64))
+    with pytest.raises(TypeError, match="w_packed"):
+        ck.linear_w4a4(x, u8.float(), bf, 64)
+    with pytest.raises(TypeError, match="bias"):
+        ck.linear_w4a4_scaled(x, u8, bf, 64, 0.5, bias=bf.half())
+    with pytest.raises(TypeError, match="wscales"):
+        ck.gemv_awq_w4a16(x[:2], u8, bf.half().reshape(2, 4), bf.reshape(2, 4))
+    with pytest.raises(TypeError, match="out"):
+        ck.gemm_w4a8_i32(i8, u8, out=torch.empty(4, 8, dtype=torch.float32))
+    with pytest.raises(ValueError, match="CUDA"):
+        ck.gemv_awq_w4a16(x[:2], u8, bf.reshape(2, 4), bf.reshape(2, 4))
