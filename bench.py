@@ -376,7 +376,8 @@ def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
         # the same product on the tcgen05 alternative (not the default path)
         ms = time_rotating(lambda c: ck.gemv_w4a8_tc(xq, xs, wps[c], sw, out=y), R, iters, 10)
         out[f"w4a8_tc_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
-                                "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R}
+                                "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R,
+                                "traffic": load_traffic("gemv_w4a8_tc_kernel")}
         del wps
     w = WL.GEMV_AWQ
     for M in w.Ms:
