@@ -94,3 +94,38 @@ def test_value_is_aggregate_units_over_slowest_rank():
     src = open(os.path.join(ROOT, "bench.py")).read()
     assert "ops * world / (ms_step * 1e-3)" in src
     assert "max_over_ranks(t[\"total_ms\"], world)" in src
+
+
+def test_traffic_entries_turn_null_when_their_kernel_sources_change(tmp_path, monkeypatch):
+    # a DRAM-traffic figure is reported only while its kernel's sources are the ones profiled
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = tmp_path / "bit_quantized_linear_rotate_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cuh").write_text("kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_source_hash(["k.cuh"])
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"k": {"source_hash": h, "dram_bytes_per_launch": 123, "sources": ["k.cuh"]}}))
+    assert bench.load_traffic("k") == 123
+    assert bench.load_traffic("missing") is None
+    (csrc / "k.cuh").write_text("kernel v2")
+    assert bench.load_traffic("k") is None
+
+
+def test_committed_traffic_entries_are_documented_and_reported_only_while_current():
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        d = json.load(f)
+    kernels = [k for k in d if not k.startswith("_")]
+    assert kernels
+    for k in kernels:
+        e = d[k]
+        assert os.path.exists(os.path.join(ROOT, e["profile"])), f"{k}: summary {e['profile']} missing"
+        assert e["dram_bytes_per_launch"] == e["read"] + e["write"]
+        current = e["source_hash"] == bench.kernel_source_hash(e["sources"])
+        assert bench.load_traffic(k) == (e["dram_bytes_per_launch"] if current else None)
