@@ -194,8 +194,22 @@ def cpu_baseline(w, rows: int, min_seconds: float = 10.0, max_passes: int = 8):
         total += oracle_linear_sample(w, rows)
         passes += 1
     ops = 2.0 * rows * w.N * w.K * passes
-    return {"value": ops / total / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {rows} of {w.M} rows of {w.name} (full K, N), {passes} passes, {total:.1f} s"}
+    out = {"value": ops / total / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"first {rows} of {w.M} rows of {w.name} (full K, N), {passes} passes, {total:.1f} s"}
+    out["single_thread"] = oracle_single_thread(w)
+    return out
+
+
+def oracle_single_thread(w, rows: int = 256):
+    """The same oracle with its BLAS limited to one thread, on a short row sample."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return None
+    with threadpool_limits(limits=1):
+        dt = oracle_linear_sample(w, rows)
+    return {"value": 2.0 * rows * w.N * w.K / dt / 1e12, "unit": "TOPS", "cores": 1,
+            "sample": f"first {rows} of {w.M} rows of {w.name}, one pass, {dt:.1f} s"}
 
 
 # ------------------------------------------------------------------ GPU legs

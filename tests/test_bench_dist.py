@@ -129,3 +129,14 @@ def test_committed_traffic_entries_are_documented_and_reported_only_while_curren
         assert e["dram_bytes_per_launch"] == e["read"] + e["write"]
         current = e["source_hash"] == bench.kernel_source_hash(e["sources"])
         assert bench.load_traffic(k) == (e["dram_bytes_per_launch"] if current else None)
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    sys.path.insert(0, ROOT)
+    import bench
+    from bit_quantized_linear_rotate_b200 import workloads as WL
+    c = bench.cpu_baseline(WL.LINEAR_M8192, rows=16, min_seconds=0.0, max_passes=1)
+    assert c["kind"] == "oracle" and c["unit"] == "TOPS" and c["value"] > 0 and c["cores"] >= 1
+    assert "16 of 8192 rows" in c["sample"]
+    st = c["single_thread"]
+    assert st is None or (st["cores"] == 1 and st["value"] > 0)
