@@ -166,6 +166,18 @@ def max_over_ranks(v: float, world: int) -> float:
     return float(t.item())
 
 
+def aggregate_e2e(e2e: dict, ops_per_step: float, world: int) -> dict:
+    """Whole-job end-to-end figure: the slowest rank's step time, the units
+    and copied bytes of all ranks (every rank feeds its own replica)."""
+    ms = max_over_ranks(e2e["ms_per_step"], world)
+    out = dict(e2e)
+    out["ms_per_step"] = ms
+    out["value"] = ops_per_step * world / (ms * 1e-3) / 1e12
+    out["h2d_bytes_per_step"] = e2e["h2d_bytes_per_step"] * world
+    out["d2h_bytes_per_step"] = e2e["d2h_bytes_per_step"] * world
+    return out
+
+
 def barrier(world: int):
     if world > 1:
         dist.barrier()
@@ -503,7 +515,9 @@ def run_ours(args, world, rank, local):
         "clocks": t["clocks"],
     }
     if not args.skip_e2e:
-        line["e2e"] = time_linear_e2e(ck, w, max(3, min(args.steps, 50)), 3, dev)
+        barrier(world)
+        e2e = time_linear_e2e(ck, w, max(3, min(args.steps, 50)), 3, dev)
+        line["e2e"] = aggregate_e2e(e2e, ops, world)
     if not args.skip_siblings:
         line["siblings"] = time_gemvs(ck, dev, peaks["hbm_gbs"])
         line["other_configs"] = time_other_configs(ck, dev, peaks)

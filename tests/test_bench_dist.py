@@ -36,12 +36,15 @@ def _rank_main(rank: int, world: int, port: int, q):
         bench.barrier(w)
         # each rank "measured" a different duration: everyone must see the slowest
         slowest = bench.max_over_ranks(10.0 + rank, w)
+        # the end-to-end figure is whole-job too: slowest rank, all ranks' units and bytes
+        e2e = bench.aggregate_e2e({"ms_per_step": 1.0 + rank, "value": 0.0, "unit": "TOPS",
+                                   "h2d_bytes_per_step": 100, "d2h_bytes_per_step": 50}, 1e12, w)
         # the reference arm prints one line on rank 0 and nothing elsewhere
         out = io.StringIO()
         with contextlib.redirect_stdout(out):
             if rank != 0:
                 bench.run_reference(type("A", (), {"warmup": 0, "steps": 1, "cpu_rows": 1})(), w, rank)
-        q.put((rank, slowest, out.getvalue()))
+        q.put((rank, slowest, out.getvalue(), e2e))
     finally:
         if dist.is_initialized():
             dist.destroy_process_group()
@@ -65,6 +68,9 @@ def test_two_rank_barrier_and_max_over_ranks():
     got = sorted(q.get(timeout=5) for _ in range(world))
     assert [g[1] for g in got] == [11.0, 11.0]
     assert got[1][2] == ""          # rank 1 printed nothing
+    for g in got:                   # 2 ranks x 1e12 ops in the slowest rank's 2 ms
+        assert g[3]["ms_per_step"] == 2.0 and abs(g[3]["value"] - 1000.0) < 1e-9
+        assert g[3]["h2d_bytes_per_step"] == 200 and g[3]["d2h_bytes_per_step"] == 100
 
 
 def test_reference_arm_prints_one_contract_line_on_rank_zero():
