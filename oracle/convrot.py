@@ -23,7 +23,7 @@ Sources (page title, then the section or symbol each function follows):
         models", Summary: ``convrot_w4a4`` and ``asym_w4a8_int8`` packed
         formats, group-size-64 ConvRot quantization.
 
-Readings where the pages are silent (each is repeated in the design doc):
+Readings where the pages are silent:
 
 * Rotation: orthonormal Sylvester Hadamard H_G / sqrt(G) applied to each
   contiguous group of G columns, y_g = x_g @ H; G = 1 is the identity
