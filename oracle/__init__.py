@@ -38,6 +38,7 @@ from .convrot import (  # noqa: F401
     hadamard_sylvester,
     int_matmul,
     linear_w4a4,
+    linear_w4a8,
     pack_nibbles,
     quantize_rowwise,
     rotate_groups,

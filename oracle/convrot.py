@@ -254,6 +254,19 @@ def linear_w4a4(x, w_packed, w_scale, G: int, bias=None, R=None, input_scale=1.0
             "y_f32": y32, "y_bits": to_bf16_bits(y32)}
 
 
+def linear_w4a8(x, w_packed, w_scale, G: int, bias=None) -> dict:
+    """ConvRot W4A8 linear ([SD] Summary, ``asym_w4a8_int8``: int4 weights against int8
+    activations): rotate + int8 quantize x (qmax 127), int matmul with the packed int4 weight,
+    the same rowwise-scale epilogue to bf16.
+
+    Returns ``q`` (M, K) int, ``s`` (M,) float32, ``acc`` (M, N) int64, ``y_f32`` and ``y_bits``.
+    """
+    q, s = rotate_quant_rowwise(x, G, 8)
+    acc = int_matmul(q, unpack_nibbles(w_packed))
+    y32 = epilogue_rowwise(acc, s, w_scale, bias)
+    return {"q": q, "s": s, "acc": acc, "y_f32": y32, "y_bits": to_bf16_bits(y32)}
+
+
 def gemv_w4a8(xq, x_scale, w_packed, w_scale, bias=None) -> dict:
     """W4A8 decode: int8 activations x int4 packed weights, same epilogue."""
     acc = int_matmul(xq, unpack_nibbles(w_packed))

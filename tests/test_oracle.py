@@ -383,3 +383,68 @@ def test_linear_w4a4_approximates_the_float_linear():
     assert rel < 0.25
     # exact identity on the quantized operands
     np.testing.assert_array_equal(O.unpack_nibbles(r["qa_packed"]), r["q"])
+
+
+# ------------------------------------------------- W4A8 linear ([SD] asym_w4a8_int8)
+
+def test_linear_w4a8_one_hot_groups_closed_form():
+    # a row that is c at the first column of every group rotates to c / sqrt(G) everywhere (the
+    # first row of the Sylvester matrix is all ones), so every int8 code is +127; weight bytes
+    # 0x00 (all nibbles u = 0, w = -8) and 0xFF (u = 15, w = 7) then give acc = 127 * w * K
+    M, K, G, c = 2, 256, 64, 3.0
+    x = np.zeros((M, K))
+    x[:, ::G] = c
+    wp = np.zeros((2, K // 2), dtype=np.uint8)
+    wp[1, :] = 0xFF
+    sw = np.full(2, 0.01, dtype=np.float32)
+    r = O.linear_w4a8(x, wp, sw, G)
+    assert np.all(r["q"] == 127)
+    np.testing.assert_array_equal(r["acc"], np.array([[-1016 * K, 889 * K]] * M))
+    s = c / np.sqrt(G) / 127
+    np.testing.assert_allclose(r["s"], s, rtol=2 ** -23)
+    y_closed = np.array([-1016 * K * s * 0.01, 889 * K * s * 0.01])
+    np.testing.assert_allclose(r["y_f32"], np.tile(y_closed, (M, 1)), rtol=1e-6)
+
+
+def test_linear_w4a8_within_half_a_code_of_the_float_linear():
+    # the stored weight lives in the rotated basis: the exact product is (x H)(sw Wq)^T, and the
+    # only error int8 activation rounding adds is at most s_m / 2 per term
+    rng = np.random.default_rng(8)
+    M, K, N, G = 6, 512, 24, 64
+    x = rng.standard_normal((M, K))
+    x[:, 5] *= 20
+    wp = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sw = rng.uniform(0.005, 0.02, N).astype(np.float32)
+    r = O.linear_w4a8(x, wp, sw, G)
+    wq = O.unpack_nibbles(wp).astype(np.float64)
+    ref = O.rotate_groups(x, G) @ (wq * sw[:, None].astype(np.float64)).T
+    bound = 0.5 * r["s"].astype(np.float64)[:, None] * (np.abs(wq).sum(axis=1) * sw)[None, :]
+    err = np.abs(r["y_f32"].astype(np.float64) - ref)
+    assert np.all(err <= bound * (1 + 1e-5) + 1e-6 * np.abs(ref))
+    # and it is far tighter than the int4 path on the same inputs (the int8 step is 127 / 7 finer)
+    r4 = O.linear_w4a4(x, wp, sw, G)
+    assert np.linalg.norm(r["y_f32"] - ref) < 0.2 * np.linalg.norm(r4["y_f32"] - ref)
+
+
+def test_linear_w4a8_brute_force_tiny():
+    # every step written out with scalar loops: closed-form Hadamard entries, Python's
+    # round-half-even, the offset-binary nibbles and the float32 epilogue products
+    rng = np.random.default_rng(9)
+    M, K, N, G = 2, 16, 3, 4
+    x = rng.standard_normal((M, K)).round(3)
+    wp = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sw = rng.uniform(0.005, 0.02, N).astype(np.float32)
+    H = [[(-1) ** bin(i & j).count("1") / G ** 0.5 for j in range(G)] for i in range(G)]
+    r = O.linear_w4a8(x, wp, sw, G)
+    for m in range(M):
+        rot = [sum(x[m, (k // G) * G + i] * H[i][k % G] for i in range(G)) for k in range(K)]
+        amax = max(abs(v) for v in rot)
+        s = np.float32(amax / 127) if amax > 0 else np.float32(1)
+        q = [max(-127, min(127, round(v / float(s)))) for v in rot]
+        assert r["q"][m].tolist() == q
+        for n in range(N):
+            w = [((int(wp[n, k // 2]) >> (4 * (k % 2))) & 0xF) - 8 for k in range(K)]
+            acc = sum(qa * wv for qa, wv in zip(q, w))
+            assert r["acc"][m, n] == acc
+            y = np.float32(np.float32(np.float32(acc) * s) * sw[n])
+            assert r["y_f32"][m, n] == y
