@@ -447,6 +447,30 @@ def time_other_configs(ck, dev, peaks):
                        "frac_int8": round(ops / (ms * 1e-3) / 1e12 / int8_peak, 4),
                        "weight_GBps": round(d["w_packed"].numel() / (ms * 1e-3) / 1e9, 1), "copies": R}
         del xs, wps
+    # the W4A8 linear (int8 activation codes) and the W4A4 linear on weights unpacked once to int8
+    # (the weight-cache trade: 2x the packed weight bytes resident, no decode in the GEMM)
+    for w in (WL.LINEAR_M8192, WL.LINEAR_MLP_DOWN):
+        d = WL.linear_inputs(w)
+        per = d["x"].numel() * 2 + 3 * d["w_packed"].numel()
+        R = max(2, -(-2 * L2_BYTES // per))
+        xs = [d["x"].to(dev) for _ in range(R)]
+        wps = [d["w_packed"].to(dev) for _ in range(R)]
+        w8s = [ck.unpack_int4(wp) for wp in wps]
+        sw = d["w_scale"].to(dev)
+        y = torch.empty(w.M, w.N, device=dev, dtype=torch.bfloat16)
+        ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
+        ops = 2.0 * w.M * w.N * w.K
+        tail = w.name.split("linear_", 1)[1]
+        for name, fn in ((f"w4a8_linear_{tail}", lambda c: ck.linear_w4a8(xs[c], wps[c], sw, w.G, workspace=ws, out=y)),
+                         (f"w4a4_linear_predecoded_{tail}",
+                          lambda c: ck.linear_w4a4_predecoded(xs[c], w8s[c], sw, w.G, workspace=ws, out=y))):
+            ms = time_rotating(fn, R, 50, 5)
+            out[name] = {"us": round(ms * 1e3, 2), "TOPS": round(ops / (ms * 1e-3) / 1e12, 1),
+                         "frac_int8": round(ops / (ms * 1e-3) / 1e12 / int8_peak, 4), "copies": R}
+            if "predecoded" in name:
+                out[name]["weight_bytes_resident"] = w.N * w.K
+                out[name]["weight_bytes_packed"] = w.N * w.K // 2
+        del xs, wps, w8s
     # rotate+quant (int8 codes, as the pages' RotateQuant measures) at the pages' activation shapes,
     # plus the MLP-down standalone case (G = 16, bits 4 and 8)
     cases = [(32, 3840, 64, 8), (8192, 3840, 64, 8), (32, 10240, 64, 8), (8192, 10240, 64, 8),

@@ -52,6 +52,10 @@ SIGNATURES = {
     "ck_linear_w4a4_scaled": [_p, _int, _i64, _i64, _i64, _i64, _int, _f32, _p, _p, _p, _p, _p, ctypes.c_size_t,
                               _p],
     "ck_linear_w4a4_static": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
+    "ck_linear_w4a8_workspace_bytes": [_i64, _i64],
+    "ck_linear_w4a8": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, ctypes.c_size_t, _p],
+    "ck_linear_w4a4_predecoded": [_p, _int, _i64, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, ctypes.c_size_t,
+                                  _p],
     "ck_gemv_w4a8": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemv_w4a8_tc": [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
     "ck_gemv_awq_w4a16": [_p, _int, _i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p],
@@ -62,7 +66,7 @@ SIGNATURES = {
     "ck_last_error": [],
     "ck_version": [],
 }
-_RESTYPES = {"ck_linear_w4a4_workspace_bytes": ctypes.c_size_t,
+_RESTYPES = {"ck_linear_w4a4_workspace_bytes": ctypes.c_size_t, "ck_linear_w4a8_workspace_bytes": ctypes.c_size_t,
              "ck_last_error": ctypes.c_char_p, "ck_version": ctypes.c_char_p}
 
 for _name, _args in SIGNATURES.items():
@@ -87,9 +91,13 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream=None):
+def _stream(stream=None, device=None):
+    """The stream handle for a call on `device`: the given stream (which must belong to that
+    device) or that device's current stream."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -120,9 +128,21 @@ def _types(where: str, **named) -> None:
 
 
 def _cuda(*ts):
+    """The one CUDA device all given tensors (None is skipped) live on; ValueError otherwise.
+
+    The library launches on the calling thread's current device, so every call below runs with
+    this device made current (``torch.cuda.device``)."""
+    dev = None
     for t in ts:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("all tensors must be CUDA tensors")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"all tensors must be on one device ({dev} and {t.device} given)")
+    return dev
 
 
 def _rows(x):
@@ -144,21 +164,35 @@ def last_error() -> str:
     return lib.ck_last_error().decode()
 
 
-def rotate_quant_rowwise(x, group_size: int, bits: int, q_out=None, scale_out=None, stream=None):
-    """Returns (q, scale): q packed int4 (..., K/2) uint8 for bits=4, int8 (..., K) for bits=8."""
-    _types("rotate_quant_rowwise", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
-    _cuda(x)
-    M, K, ldx, x2 = _rows(x)
+def _call(dev, name: str, *args, stream=None) -> None:
+    """Calls the C entry point `name` with `dev` current and that device's stream appended."""
+    with torch.cuda.device(dev):
+        _check(getattr(lib, name)(*args, _stream(stream, dev)), name)
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _codes_out(x, K, bits, q_out, scale_out):
     lead = tuple(x.shape[:-1])
     if q_out is None:
         q_out = torch.empty(lead + ((K // 2,) if bits == 4 else (K,)), device=x.device,
                             dtype=torch.uint8 if bits == 4 else torch.int8)
     if scale_out is None:
         scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
-    _cuda(q_out, scale_out)
-    _check(lib.ck_rotate_quant_rowwise(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
-                                       _ptr(q_out), _ptr(scale_out), _stream(stream)),
-           "ck_rotate_quant_rowwise")
+    return q_out, scale_out
+
+
+def rotate_quant_rowwise(x, group_size: int, bits: int, q_out=None, scale_out=None, stream=None):
+    """Returns (q, scale): q packed int4 (..., K/2) uint8 for bits=4, int8 (..., K) for bits=8."""
+    _types("rotate_quant_rowwise", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
+    _cuda(x)
+    M, K, ldx, x2 = _rows(x)
+    q_out, scale_out = _codes_out(x, K, bits, q_out, scale_out)
+    dev = _cuda(x, q_out, scale_out)
+    _call(dev, "ck_rotate_quant_rowwise", _ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
+          _ptr(q_out), _ptr(scale_out), stream=stream)
     return q_out, scale_out
 
 
@@ -167,15 +201,10 @@ def rotate_quant_rowwise_i8(x, group_size: int, bits: int, q_out=None, scale_out
     _types("rotate_quant_rowwise_i8", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
     _cuda(x)
     M, K, ldx, x2 = _rows(x)
-    lead = tuple(x.shape[:-1])
-    if q_out is None:
-        q_out = torch.empty(lead + (K,), device=x.device, dtype=torch.int8)
-    if scale_out is None:
-        scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
-    _cuda(q_out, scale_out)
-    _check(lib.ck_rotate_quant_rowwise_i8(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
-                                          _ptr(q_out), _ptr(scale_out), _stream(stream)),
-           "ck_rotate_quant_rowwise_i8")
+    q_out, scale_out = _codes_out(x, K, 8, q_out, scale_out)
+    dev = _cuda(x, q_out, scale_out)
+    _call(dev, "ck_rotate_quant_rowwise_i8", _ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
+          _ptr(q_out), _ptr(scale_out), stream=stream)
     return q_out, scale_out
 
 
@@ -190,15 +219,10 @@ def rotate_quant_rowwise_r(x, R, bits: int, q_out=None, scale_out=None, stream=N
     if R.dtype != torch.float32 or R.dim() != 2 or R.shape[0] != R.shape[1] or not R.is_contiguous():
         raise ValueError("R must be a contiguous square float32 matrix")
     M, K, ldx, x2 = _rows(x)
-    lead = tuple(x.shape[:-1])
-    if q_out is None:
-        q_out = torch.empty(lead + ((K // 2,) if bits == 4 else (K,)), device=x.device,
-                            dtype=torch.uint8 if bits == 4 else torch.int8)
-    if scale_out is None:
-        scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
-    _check(lib.ck_rotate_quant_rowwise_r(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, R.shape[0], _ptr(R), bits,
-                                         _ptr(q_out), _ptr(scale_out), _stream(stream)),
-           "ck_rotate_quant_rowwise_r")
+    q_out, scale_out = _codes_out(x, K, bits, q_out, scale_out)
+    dev = _cuda(x, R, q_out, scale_out)
+    _call(dev, "ck_rotate_quant_rowwise_r", _ptr(x2), _dtype_code(x.dtype), M, K, ldx, R.shape[0], _ptr(R), bits,
+          _ptr(q_out), _ptr(scale_out), stream=stream)
     return q_out, scale_out
 
 
@@ -208,16 +232,10 @@ def rotate_quant_rowwise_scaled(x, group_size: int, bits: int, input_scale: floa
     _types("rotate_quant_rowwise_scaled", x=(x, _HALF), q_out=(q_out, _BYTES), scale_out=(scale_out, _F32))
     _cuda(x)
     M, K, ldx, x2 = _rows(x)
-    lead = tuple(x.shape[:-1])
-    if q_out is None:
-        q_out = torch.empty(lead + ((K // 2,) if bits == 4 else (K,)), device=x.device,
-                            dtype=torch.uint8 if bits == 4 else torch.int8)
-    if scale_out is None:
-        scale_out = torch.empty(lead, device=x.device, dtype=torch.float32)
-    _cuda(q_out, scale_out)
-    _check(lib.ck_rotate_quant_rowwise_scaled(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
-                                              float(input_scale), _ptr(q_out), _ptr(scale_out), _stream(stream)),
-           "ck_rotate_quant_rowwise_scaled")
+    q_out, scale_out = _codes_out(x, K, bits, q_out, scale_out)
+    dev = _cuda(x, q_out, scale_out)
+    _call(dev, "ck_rotate_quant_rowwise_scaled", _ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, bits,
+          float(input_scale), _ptr(q_out), _ptr(scale_out), stream=stream)
     return q_out, scale_out
 
 
@@ -228,58 +246,59 @@ def unpack_int4(packed, out=None, stream=None):
     R, Ch = packed.shape
     if out is None:
         out = torch.empty((R, 2 * Ch), device=packed.device, dtype=torch.int8)
-    _check(lib.ck_unpack_int4(_ptr(packed), R, 2 * Ch, _ptr(out), _stream(stream)), "ck_unpack_int4")
+    dev = _cuda(packed, out)
+    _call(dev, "ck_unpack_int4", _ptr(packed), R, 2 * Ch, _ptr(out), stream=stream)
     return out
+
+
+def _mn_out(a, M, N, out, dtype=torch.bfloat16):
+    return torch.empty((M, N), device=a.device, dtype=dtype) if out is None else out
 
 
 def gemm_w4a8(qa, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):
     """int8 activation codes (M, K) x packed int4 weights (N, K/2) -> bf16 (M, N)."""
     _types("gemm_w4a8", qa=(qa, _BYTES), a_scale=(a_scale, _F32), w_packed=(w_packed, _BYTES),
            w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
-    _cuda(qa, a_scale, w_packed, w_scale, bias)
+    _cuda(qa, a_scale, w_packed, w_scale, bias, out)
     M, K = qa.shape
     N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=qa.device, dtype=torch.bfloat16)
-    _check(lib.ck_gemm_w4a8(_ptr(qa), _ptr(a_scale), M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias),
-                            _ptr(out), _stream(stream)), "ck_gemm_w4a8")
+    out = _mn_out(qa, M, N, out)
+    _call(_cuda(qa, out), "ck_gemm_w4a8", _ptr(qa), _ptr(a_scale), M, K, N, _ptr(w_packed), _ptr(w_scale),
+          _ptr(bias), _ptr(out), stream=stream)
     return out
 
 
 def gemm_s8(qa, a_scale, w8, w_scale, bias=None, out=None, stream=None):
     _types("gemm_s8", qa=(qa, _BYTES), a_scale=(a_scale, _F32), w8=(w8, _BYTES), w_scale=(w_scale, _BF16),
            bias=(bias, _BF16), out=(out, _BF16))
-    _cuda(qa, a_scale, w8, w_scale, bias)
+    _cuda(qa, a_scale, w8, w_scale, bias, out)
     M, K = qa.shape
     N = w8.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=qa.device, dtype=torch.bfloat16)
-    _check(lib.ck_gemm_s8(_ptr(qa), _ptr(a_scale), M, K, N, _ptr(w8), _ptr(w_scale), _ptr(bias), _ptr(out),
-                          _stream(stream)), "ck_gemm_s8")
+    out = _mn_out(qa, M, N, out)
+    _call(_cuda(qa, out), "ck_gemm_s8", _ptr(qa), _ptr(a_scale), M, K, N, _ptr(w8), _ptr(w_scale), _ptr(bias),
+          _ptr(out), stream=stream)
     return out
 
 
 def gemm_s8_i32(qa, w8, out=None, stream=None):
     _types("gemm_s8_i32", qa=(qa, _BYTES), w8=(w8, _BYTES), out=(out, _I32))
-    _cuda(qa, w8)
+    _cuda(qa, w8, out)
     M, K = qa.shape
     N = w8.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=qa.device, dtype=torch.int32)
-    _check(lib.ck_gemm_s8_i32(_ptr(qa), _ptr(w8), M, K, N, _ptr(out), _stream(stream)), "ck_gemm_s8_i32")
+    out = _mn_out(qa, M, N, out, torch.int32)
+    _call(_cuda(qa, out), "ck_gemm_s8_i32", _ptr(qa), _ptr(w8), M, K, N, _ptr(out), stream=stream)
     return out
 
 
 def gemm_w4a4(qa_packed, a_scale, w_packed, w_scale, bias=None, out=None, stream=None):
     _types("gemm_w4a4", qa_packed=(qa_packed, _BYTES), a_scale=(a_scale, _F32), w_packed=(w_packed, _BYTES),
            w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
-    _cuda(qa_packed, a_scale, w_packed, w_scale, bias)
+    _cuda(qa_packed, a_scale, w_packed, w_scale, bias, out)
     M, Kh = qa_packed.shape
     N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=qa_packed.device, dtype=torch.bfloat16)
-    _check(lib.ck_gemm_w4a4(_ptr(qa_packed), _ptr(a_scale), M, 2 * Kh, N, _ptr(w_packed), _ptr(w_scale),
-                            _ptr(bias), _ptr(out), _stream(stream)), "ck_gemm_w4a4")
+    out = _mn_out(qa_packed, M, N, out)
+    _call(_cuda(qa_packed, out), "ck_gemm_w4a4", _ptr(qa_packed), _ptr(a_scale), M, 2 * Kh, N, _ptr(w_packed),
+          _ptr(w_scale), _ptr(bias), _ptr(out), stream=stream)
     return out
 
 
@@ -287,44 +306,53 @@ def linear_w4a4_workspace_bytes(M: int, K: int) -> int:
     return int(lib.ck_linear_w4a4_workspace_bytes(M, K))
 
 
+def linear_w4a8_workspace_bytes(M: int, K: int) -> int:
+    return int(lib.ck_linear_w4a8_workspace_bytes(M, K))
+
+
+def _linear(name, x, w, w_scale, group_size, bias, workspace, out, stream, ws_fn, *extra, w_name="w_packed"):
+    """Shared marshalling of the one-shot linears: (x, weights, scales) -> y (..., N) bf16."""
+    _types(name, x=(x, _HALF), **{w_name: (w, _BYTES)}, w_scale=(w_scale, _BF16), bias=(bias, _BF16),
+           out=(out, _BF16), workspace=(workspace, _BYTES))
+    _cuda(x, w, w_scale, bias, workspace, out)
+    M, K, ldx, x2 = _rows(x)
+    N = w.shape[0]
+    if workspace is None:
+        workspace = torch.empty(ws_fn(M, K), device=x.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), device=x.device, dtype=torch.bfloat16)
+    dev = _cuda(x, workspace, out)
+    _call(dev, "ck_" + name, _ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size, *extra, _ptr(w),
+          _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace), _nbytes(workspace), stream=stream)
+    return out
+
+
 def linear_w4a4(x, w_packed, w_scale, group_size: int, bias=None, workspace=None, out=None,
                 stream=None):
     """ConvRot W4A4 linear: y (..., N) bf16 from x (..., K) bf16/fp16 and packed (N, K/2) weights."""
-    _types("linear_w4a4", x=(x, _HALF), w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
-           out=(out, _BF16))
-    _cuda(x, w_packed, w_scale, bias)
-    M, K, ldx, x2 = _rows(x)
-    N = w_packed.shape[0]
-    ws_bytes = linear_w4a4_workspace_bytes(M, K)
-    if workspace is None:
-        workspace = torch.empty(ws_bytes, device=x.device, dtype=torch.uint8)
-    if out is None:
-        out = torch.empty(tuple(x.shape[:-1]) + (N,), device=x.device, dtype=torch.bfloat16)
-    _check(lib.ck_linear_w4a4(_ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size, _ptr(w_packed),
-                              _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _stream(stream)),
-           "ck_linear_w4a4")
-    return out
+    return _linear("linear_w4a4", x, w_packed, w_scale, group_size, bias, workspace, out, stream,
+                   linear_w4a4_workspace_bytes)
+
+
+def linear_w4a8(x, w_packed, w_scale, group_size: int, bias=None, workspace=None, out=None,
+                stream=None):
+    """ConvRot W4A8 linear: x rotated and quantized to int8 codes, times packed (N, K/2) int4 weights."""
+    return _linear("linear_w4a8", x, w_packed, w_scale, group_size, bias, workspace, out, stream,
+                   linear_w4a8_workspace_bytes)
+
+
+def linear_w4a4_predecoded(x, w_s8, w_scale, group_size: int, bias=None, workspace=None, out=None,
+                           stream=None):
+    """linear_w4a4 with the weights already unpacked to int8 (N, K) by unpack_int4 (same results)."""
+    return _linear("linear_w4a4_predecoded", x, w_s8, w_scale, group_size, bias, workspace, out, stream,
+                   linear_w4a4_workspace_bytes, w_name="w_s8")
 
 
 def linear_w4a4_scaled(x, w_packed, w_scale, group_size: int, input_scale: float, bias=None, workspace=None,
                        out=None, stream=None):
     """linear_w4a4 of input_scale * x (a finite tensor-wise scale >= 0); the output is not rescaled."""
-    _types("linear_w4a4_scaled", x=(x, _HALF), w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
-           out=(out, _BF16))
-    _cuda(x, w_packed, w_scale, bias)
-    M, K, ldx, x2 = _rows(x)
-    N = w_packed.shape[0]
-    ws_bytes = linear_w4a4_workspace_bytes(M, K)
-    if workspace is None:
-        workspace = torch.empty(ws_bytes, device=x.device, dtype=torch.uint8)
-    if out is None:
-        out = torch.empty(tuple(x.shape[:-1]) + (N,), device=x.device, dtype=torch.bfloat16)
-    _check(lib.ck_linear_w4a4_scaled(_ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size, float(input_scale),
-                                     _ptr(w_packed), _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(workspace),
-                                     workspace.numel() * workspace.element_size(), _stream(stream)),
-           "ck_linear_w4a4_scaled")
-    return out
+    return _linear("linear_w4a4_scaled", x, w_packed, w_scale, group_size, bias, workspace, out, stream,
+                   linear_w4a4_workspace_bytes, ctypes.c_float(float(input_scale)))
 
 
 # Size of the library's built-in scratch for linear_w4a4_static (CK_LINEAR_STATIC_SCRATCH_BYTES).
@@ -335,71 +363,62 @@ def linear_w4a4_static(x, w_packed, w_scale, group_size: int, bias=None, out=Non
     """linear_w4a4 without a workspace argument: the library uses its own fixed per-device scratch.
 
     Same results as linear_w4a4. Calls on one device share that scratch, so calls that may run
-    at the same time on the GPU (different streams, several threads) must not be mixed.
+    at the same time on the GPU (different streams, several threads) must not be mixed. The call
+    runs with x's device current: the scratch it uses is that device's.
     """
-    _types("linear_w4a4_static", x=(x, _HALF), w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
-           out=(out, _BF16))
-    _cuda(x, w_packed, w_scale, bias)
+    _types("linear_w4a4_static", x=(x, _HALF), w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16),
+           bias=(bias, _BF16), out=(out, _BF16))
+    _cuda(x, w_packed, w_scale, bias, out)
     M, K, ldx, x2 = _rows(x)
     N = w_packed.shape[0]
     if out is None:
         out = torch.empty(tuple(x.shape[:-1]) + (N,), device=x.device, dtype=torch.bfloat16)
-    _check(lib.ck_linear_w4a4_static(_ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size, _ptr(w_packed),
-                                     _ptr(w_scale), _ptr(bias), _ptr(out), _stream(stream)),
-           "ck_linear_w4a4_static")
+    _call(_cuda(x, out), "ck_linear_w4a4_static", _ptr(x2), _dtype_code(x.dtype), M, K, N, ldx, group_size,
+          _ptr(w_packed), _ptr(w_scale), _ptr(bias), _ptr(out), stream=stream)
     return out
 
 
 def linear_w4a4_quantize(x, group_size: int, workspace, stream=None):
     """Phase 1 of linear_w4a4: rotate + quantize x into `workspace` (opaque)."""
-    _types("linear_w4a4_quantize", x=(x, _HALF))
-    _cuda(x, workspace)
+    _types("linear_w4a4_quantize", x=(x, _HALF), workspace=(workspace, _BYTES))
+    dev = _cuda(x, workspace)
     M, K, ldx, x2 = _rows(x)
-    _check(lib.ck_linear_w4a4_quantize(_ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, _ptr(workspace),
-                                       workspace.numel() * workspace.element_size(), _stream(stream)),
-           "ck_linear_w4a4_quantize")
+    _call(dev, "ck_linear_w4a4_quantize", _ptr(x2), _dtype_code(x.dtype), M, K, ldx, group_size, _ptr(workspace),
+          _nbytes(workspace), stream=stream)
     return workspace
 
 
 def linear_w4a4_matmul(M: int, K: int, w_packed, w_scale, workspace, bias=None, out=None, stream=None):
     """Phase 2 of linear_w4a4: GEMM of the workspace codes with the packed weights -> y (M, N) bf16."""
     _types("linear_w4a4_matmul", w_packed=(w_packed, _BYTES), w_scale=(w_scale, _BF16), bias=(bias, _BF16),
-           out=(out, _BF16))
-    _cuda(w_packed, w_scale, workspace, bias)
+           out=(out, _BF16), workspace=(workspace, _BYTES))
+    _cuda(w_packed, w_scale, workspace, bias, out)
     N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=w_packed.device, dtype=torch.bfloat16)
-    _check(lib.ck_linear_w4a4_matmul(M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias), _ptr(out),
-                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                     _stream(stream)), "ck_linear_w4a4_matmul")
+    out = _mn_out(w_packed, M, N, out)
+    _call(_cuda(w_packed, workspace, out), "ck_linear_w4a4_matmul", M, K, N, _ptr(w_packed), _ptr(w_scale),
+          _ptr(bias), _ptr(out), _ptr(workspace), _nbytes(workspace), stream=stream)
+    return out
+
+
+def _gemv_w4a8(name, xq, x_scale, w_packed, w_scale, bias, out, stream):
+    _types(name, xq=(xq, _BYTES), x_scale=(x_scale, _F32), w_packed=(w_packed, _BYTES),
+           w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
+    _cuda(xq, x_scale, w_packed, w_scale, bias, out)
+    M, K = xq.shape
+    N = w_packed.shape[0]
+    out = _mn_out(xq, M, N, out)
+    _call(_cuda(xq, out), "ck_" + name, _ptr(xq), _ptr(x_scale), M, K, N, _ptr(w_packed), _ptr(w_scale),
+          _ptr(bias), _ptr(out), stream=stream)
     return out
 
 
 def gemv_w4a8(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
-    _types("gemv_w4a8", xq=(xq, _BYTES), x_scale=(x_scale, _F32), w_packed=(w_packed, _BYTES),
-           w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
-    _cuda(xq, x_scale, w_packed, w_scale, bias)
-    M, K = xq.shape
-    N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=xq.device, dtype=torch.bfloat16)
-    _check(lib.ck_gemv_w4a8(_ptr(xq), _ptr(x_scale), M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias),
-                            _ptr(out), _stream(stream)), "ck_gemv_w4a8")
-    return out
+    return _gemv_w4a8("gemv_w4a8", xq, x_scale, w_packed, w_scale, bias, out, stream)
 
 
 def gemv_w4a8_tc(xq, x_scale, w_packed, w_scale, bias=None, out=None, stream=None):
     """gemv_w4a8 on the tcgen05 tensor cores (the same results bit for bit; an alternative path)."""
-    _types("gemv_w4a8_tc", xq=(xq, _BYTES), x_scale=(x_scale, _F32), w_packed=(w_packed, _BYTES),
-           w_scale=(w_scale, _BF16), bias=(bias, _BF16), out=(out, _BF16))
-    _cuda(xq, x_scale, w_packed, w_scale, bias)
-    M, K = xq.shape
-    N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=xq.device, dtype=torch.bfloat16)
-    _check(lib.ck_gemv_w4a8_tc(_ptr(xq), _ptr(x_scale), M, K, N, _ptr(w_packed), _ptr(w_scale), _ptr(bias),
-                               _ptr(out), _stream(stream)), "ck_gemv_w4a8_tc")
-    return out
+    return _gemv_w4a8("gemv_w4a8_tc", xq, x_scale, w_packed, w_scale, bias, out, stream)
 
 
 def gemv_awq_w4a16(x, qweight, wscales, wzeros, bias=None, group_size: int = 64, out=None, stream=None):
@@ -407,38 +426,33 @@ def gemv_awq_w4a16(x, qweight, wscales, wzeros, bias=None, group_size: int = 64,
     same = (x.dtype,) if x.dtype in _HALF else _HALF
     _types("gemv_awq_w4a16", x=(x, _HALF), qweight=(qweight, _BYTES), wscales=(wscales, same),
            wzeros=(wzeros, same), bias=(bias, same), out=(out, same))
-    _cuda(x, qweight, wscales, wzeros, bias)
+    _cuda(x, qweight, wscales, wzeros, bias, out)
     M, K = x.shape
     N = qweight.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=x.device, dtype=x.dtype)
-    _check(lib.ck_gemv_awq_w4a16(_ptr(x), _dtype_code(x.dtype), M, K, N, group_size, _ptr(qweight),
-                                 _ptr(wscales), _ptr(wzeros), _ptr(bias), _ptr(out), _stream(stream)),
-           "ck_gemv_awq_w4a16")
+    out = _mn_out(x, M, N, out, x.dtype)
+    _call(_cuda(x, out), "ck_gemv_awq_w4a16", _ptr(x), _dtype_code(x.dtype), M, K, N, group_size, _ptr(qweight),
+          _ptr(wscales), _ptr(wzeros), _ptr(bias), _ptr(out), stream=stream)
     return out
 
 
 def gemm_w4a4_i32(qa_packed, w_packed, out=None, stream=None):
     _types("gemm_w4a4_i32", qa_packed=(qa_packed, _BYTES), w_packed=(w_packed, _BYTES), out=(out, _I32))
-    _cuda(qa_packed, w_packed)
+    _cuda(qa_packed, w_packed, out)
     M, Kh = qa_packed.shape
     N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=qa_packed.device, dtype=torch.int32)
-    _check(lib.ck_gemm_w4a4_i32(_ptr(qa_packed), _ptr(w_packed), M, 2 * Kh, N, _ptr(out), _stream(stream)),
-           "ck_gemm_w4a4_i32")
+    out = _mn_out(qa_packed, M, N, out, torch.int32)
+    _call(_cuda(qa_packed, out), "ck_gemm_w4a4_i32", _ptr(qa_packed), _ptr(w_packed), M, 2 * Kh, N, _ptr(out),
+          stream=stream)
     return out
 
 
 def gemm_w4a8_i32(qa, w_packed, out=None, stream=None):
     _types("gemm_w4a8_i32", qa=(qa, _BYTES), w_packed=(w_packed, _BYTES), out=(out, _I32))
-    _cuda(qa, w_packed)
+    _cuda(qa, w_packed, out)
     M, K = qa.shape
     N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), device=qa.device, dtype=torch.int32)
-    _check(lib.ck_gemm_w4a8_i32(_ptr(qa), _ptr(w_packed), M, K, N, _ptr(out), _stream(stream)),
-           "ck_gemm_w4a8_i32")
+    out = _mn_out(qa, M, N, out, torch.int32)
+    _call(_cuda(qa, out), "ck_gemm_w4a8_i32", _ptr(qa), _ptr(w_packed), M, K, N, _ptr(out), stream=stream)
     return out
 
 

@@ -294,13 +294,14 @@ void launch_rq_store(int bits, int store, const void* x, int64_t M, int K, int64
                      float* s, int32_t* rs, int nt, float a, cudaStream_t st) {
   using namespace ck::rq;
   if (store == STORE_PACKED4) launch_rq<4, STORE_PACKED4, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
-  else if (store == STORE_INT8_PERM) launch_rq<4, STORE_INT8_PERM, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
+  else if (store == STORE_INT8_PERM && bits == 4) launch_rq<4, STORE_INT8_PERM, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
+  else if (store == STORE_INT8_PERM) launch_rq<8, STORE_INT8_PERM, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
   else if (bits == 4) launch_rq<4, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
   else launch_rq<8, STORE_INT8, T>(x, M, K, ldx, G, q, s, rs, nt, a, st);
 }
 
 // store: STORE_PACKED4 (bits 4), STORE_INT8 (codes as int8 bytes) or STORE_INT8_PERM
-// (bits 4, the linear's GEMM-ready activations with row sums in `rs`). in_scale:
+// (bits 4 or 8, the linears' GEMM-ready activations with row sums in `rs`). in_scale:
 // the tensor-wise input scale, validated by the caller (finite, >= 0, 1 when G = 1).
 ck_status rotate_quant_impl(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int G,
                             int bits, int store, void* q, float* s, int32_t* rs, cudaStream_t st,
@@ -656,9 +657,18 @@ size_t ck_linear_w4a4_workspace_bytes(int64_t M, int64_t K) {
 
 namespace {
 
+// The linears' activation code widths: int4 codes (the W4A4 linear) or int8
+// codes (the W4A8 linear); the GEMM multiplies either with unsigned nibbles.
+int64_t linear_term(int bits) { return bits == 4 ? kTermLinear : kTermGemv; }
+
+// Phase 1 of a linear: rotate + quantize x into the workspace. `perm` selects
+// the GEMM-ready format (codes in permuted column order plus row sums, for the
+// tensor-core GEMM with unsigned weight decode); otherwise the codes stay in
+// natural order (the decode-GEMV route and the pre-decoded-weight GEMM).
 ck_status linear_quantize_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
-                                int group_size, float in_scale, void* workspace, size_t ws_bytes, void* stream) {
-  ck_status r = check_gemm_shape(who, M, K, 1, kTermLinear);
+                                int group_size, int bits, float in_scale, bool perm, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  ck_status r = check_gemm_shape(who, M, K, 1, linear_term(bits));
   if (r != CK_OK) return r;
   if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
   if (xt != CK_BF16 && xt != CK_FP16) return fail(CK_ERR_INVALID_ARG, "%s: unknown dtype", who);
@@ -670,31 +680,23 @@ ck_status linear_quantize_entry(const char* who, const void* x, ck_dtype xt, int
   if (x == nullptr) return fail(CK_ERR_INVALID_ARG, "%s: null pointer", who);
   if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "%s: x rows must be 16-byte aligned", who);
   LinearWs ws = linear_ws(workspace, M, K);
-  const int store = linear_small_m(M, K) ? ck::rq::STORE_INT8 : ck::rq::STORE_INT8_PERM;
-  return rotate_quant_impl(x, xt, M, K, ldx, group_size, 4, store, ws.q, ws.scale, ws.rowsum, S(stream),
+  const int store = perm ? ck::rq::STORE_INT8_PERM : ck::rq::STORE_INT8;
+  return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, store, ws.q, ws.scale, ws.rowsum, S(stream),
                            in_scale);
 }
 
-}  // namespace
-
-extern "C" {
-
-ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int group_size,
-                                  void* workspace, size_t ws_bytes, void* stream) {
-  return linear_quantize_entry("linear_w4a4_quantize", x, xt, M, K, ldx, group_size, 1.0f, workspace, ws_bytes,
-                               stream);
-}
-
-ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
-                                const uint16_t* bias, uint16_t* y, const void* workspace, size_t ws_bytes,
-                                void* stream) {
-  ck_status r = check_gemm_shape("linear_w4a4_matmul", M, K, N, kTermLinear);
+// Phase 2 of a linear on packed int4 weights: the small-batch decode GEMV or
+// the tensor-core GEMM with unsigned weight decode, on the codes phase 1 wrote.
+ck_status linear_matmul_entry(const char* who, int64_t M, int64_t K, int64_t N, int bits, const uint8_t* w_packed,
+                              const uint16_t* w_scale, const uint16_t* bias, uint16_t* y, const void* workspace,
+                              size_t ws_bytes, void* stream) {
+  ck_status r = check_gemm_shape(who, M, K, N, linear_term(bits));
   if (r != CK_OK) return r;
-  if ((r = check_linear_workspace("linear_w4a4_matmul", M, K, workspace, ws_bytes)) != CK_OK) return r;
-  if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_matmul: null pointer");
-  if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "linear_w4a4_matmul: weights must be 16-byte aligned");
+  if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
+  if (!w_packed || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "%s: weights must be 16-byte aligned", who);
   if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
-    return fail(CK_ERR_INVALID_ARG, "linear_w4a4_matmul: misaligned scale, bias or output");
+    return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
   LinearWs ws = linear_ws(const_cast<void*>(workspace), M, K);
   if (linear_small_m(M, K)) {
     for (int64_t r0 = 0; r0 < M; r0 += kSmallMChunk) {
@@ -708,14 +710,31 @@ ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* 
       ws.q, M, K, N, w_packed, ws.scale, ws.rowsum, w_scale, bias, y, S(stream));
 }
 
+}  // namespace
+
+extern "C" {
+
+ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int group_size,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  return linear_quantize_entry("linear_w4a4_quantize", x, xt, M, K, ldx, group_size, 4, 1.0f,
+                               !linear_small_m(M, K), workspace, ws_bytes, stream);
+}
+
+ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
+                                const uint16_t* bias, uint16_t* y, const void* workspace, size_t ws_bytes,
+                                void* stream) {
+  return linear_matmul_entry("linear_w4a4_matmul", M, K, N, 4, w_packed, w_scale, bias, y, workspace, ws_bytes,
+                             stream);
+}
+
 }  // extern "C"
 
 namespace {
 
 ck_status linear_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
-                       int group_size, float in_scale, const uint8_t* w_packed, const uint16_t* w_scale,
+                       int group_size, int bits, float in_scale, const uint8_t* w_packed, const uint16_t* w_scale,
                        const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
-  ck_status r = check_gemm_shape(who, M, K, N, kTermLinear);
+  ck_status r = check_gemm_shape(who, M, K, N, linear_term(bits));
   if (r != CK_OK) return r;
   // validate both phases before enqueuing either
   if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
@@ -723,9 +742,10 @@ ck_status linear_entry(const char* who, const void* x, ck_dtype xt, int64_t M, i
   if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "%s: weights must be 16-byte aligned", who);
   if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
-  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, in_scale, workspace, ws_bytes, stream);
+  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, bits, in_scale, !linear_small_m(M, K), workspace,
+                            ws_bytes, stream);
   if (r != CK_OK) return r;
-  return ck_linear_w4a4_matmul(M, K, N, w_packed, w_scale, bias, y, workspace, ws_bytes, stream);
+  return linear_matmul_entry(who, M, K, N, bits, w_packed, w_scale, bias, y, workspace, ws_bytes, stream);
 }
 
 }  // namespace
@@ -736,7 +756,7 @@ ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64
                          int group_size, const uint8_t* w_packed, const uint16_t* w_scale,
                          const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes,
                          void* stream) {
-  return linear_entry("linear_w4a4", x, xt, M, K, N, ldx, group_size, 1.0f, w_packed, w_scale, bias, y,
+  return linear_entry("linear_w4a4", x, xt, M, K, N, ldx, group_size, 4, 1.0f, w_packed, w_scale, bias, y,
                       workspace, ws_bytes, stream);
 }
 
@@ -744,8 +764,37 @@ ck_status ck_linear_w4a4_scaled(const void* x, ck_dtype xt, int64_t M, int64_t K
                                 int group_size, float input_scale, const uint8_t* w_packed,
                                 const uint16_t* w_scale, const uint16_t* bias, uint16_t* y, void* workspace,
                                 size_t ws_bytes, void* stream) {
-  return linear_entry("linear_w4a4_scaled", x, xt, M, K, N, ldx, group_size, input_scale, w_packed, w_scale,
+  return linear_entry("linear_w4a4_scaled", x, xt, M, K, N, ldx, group_size, 4, input_scale, w_packed, w_scale,
                       bias, y, workspace, ws_bytes, stream);
+}
+
+size_t ck_linear_w4a8_workspace_bytes(int64_t M, int64_t K) { return ck_linear_w4a4_workspace_bytes(M, K); }
+
+ck_status ck_linear_w4a8(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
+                         int group_size, const uint8_t* w_packed, const uint16_t* w_scale,
+                         const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  return linear_entry("linear_w4a8", x, xt, M, K, N, ldx, group_size, 8, 1.0f, w_packed, w_scale, bias, y,
+                      workspace, ws_bytes, stream);
+}
+
+ck_status ck_linear_w4a4_predecoded(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N, int64_t ldx,
+                                    int group_size, const int8_t* w_s8, const uint16_t* w_scale,
+                                    const uint16_t* bias, uint16_t* y, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  const char* who = "linear_w4a4_predecoded";
+  ck_status r = check_gemm_shape(who, M, K, N, kTermLinear);
+  if (r != CK_OK) return r;
+  if ((r = check_linear_workspace(who, M, K, workspace, ws_bytes)) != CK_OK) return r;
+  if (!w_s8 || !w_scale || !y) return fail(CK_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!aligned(w_s8, 16)) return fail(CK_ERR_UNSUPPORTED, "%s: weights must be 16-byte aligned", who);
+  if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
+    return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
+  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, 4, 1.0f, false, workspace, ws_bytes, stream);
+  if (r != CK_OK) return r;
+  LinearWs ws = linear_ws(workspace, M, K);
+  return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_BF16>(
+      ws.q, M, K, N, w_s8, ws.scale, nullptr, w_scale, bias, y, S(stream));
 }
 
 }  // extern "C"
@@ -761,27 +810,68 @@ namespace {
 
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxScratchDevices] = {};
+struct ScratchEntry {
+  void* addr;   // device address of g_linear_scratch
+  void* ctx;    // the context it was looked up in
+};
+ScratchEntry g_scratch[kMaxScratchDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The calling thread's current CUDA context (null if it cannot be read).
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return reinterpret_cast<void*>(c);
+}
 
 // Device address of g_linear_scratch on the current device, looked up on the
-// first call for that device and cached.
-ck_status static_scratch_addr(void** out) {
+// first call for that device and cached together with the current context; a
+// different context (the device was reset and its context made anew, say)
+// triggers a new lookup, since the module, and the array with it, was loaded
+// again. Fails if `x` does not live on the current device, whose scratch the
+// call would otherwise pair with another device's data.
+ck_status static_scratch_addr(const void* x, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess)
     return fail(CK_ERR_CUDA, "linear_w4a4_static: cudaGetDevice failed: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxScratchDevices)
     return fail(CK_ERR_UNSUPPORTED, "linear_w4a4_static: device ordinal %d >= %d", dev, kMaxScratchDevices);
+  cudaPointerAttributes pa;
+  e = cudaPointerGetAttributes(&pa, x);
+  if (e != cudaSuccess) {
+    cudaGetLastError();   // clear the error this records, so that a later launch check does not see it
+    return fail(CK_ERR_INVALID_ARG, "linear_w4a4_static: x is not a device pointer (%s)", cudaGetErrorString(e));
+  }
+  if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
+    return fail(CK_ERR_INVALID_ARG, "linear_w4a4_static: x is not device memory");
+  if (pa.device != dev)
+    return fail(CK_ERR_INVALID_ARG,
+                "linear_w4a4_static: x is on device %d but device %d is current; make x's device current",
+                pa.device, dev);
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchEntry& ent = g_scratch[dev];
+  if (ent.addr == nullptr || ent.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_linear_scratch);
     if (e != cudaSuccess || p == nullptr)
       return fail(CK_ERR_CUDA, "linear_w4a4_static: cudaGetSymbolAddress failed on device %d: %s", dev,
                   cudaGetErrorString(e));
-    g_scratch_addr[dev] = p;
+    ent.addr = p;
+    ent.ctx = ctx;
   }
-  *out = g_scratch_addr[dev];
+  *out = ent.addr;
   return CK_OK;
 }
 
@@ -801,8 +891,9 @@ ck_status ck_linear_w4a4_static(const void* x, ck_dtype xt, int64_t M, int64_t K
                 "linear_w4a4_static: M=%lld, K=%lld need %zu bytes of scratch, more than the %zu-byte "
                 "static scratch; call ck_linear_w4a4 with a workspace instead",
                 (long long)M, (long long)K, need, (size_t)CK_LINEAR_STATIC_SCRATCH_BYTES);
+  if (x == nullptr) return fail(CK_ERR_INVALID_ARG, "linear_w4a4_static: null pointer");
   void* scratch = nullptr;
-  if ((r = static_scratch_addr(&scratch)) != CK_OK) return r;
+  if ((r = static_scratch_addr(x, &scratch)) != CK_OK) return r;
   return ck_linear_w4a4(x, xt, M, K, N, ldx, group_size, w_packed, w_scale, bias, y, scratch,
                         (size_t)CK_LINEAR_STATIC_SCRATCH_BYTES, stream);
 }

@@ -232,6 +232,50 @@ ck_status ck_linear_w4a4_scaled(const void* x, ck_dtype xt, int64_t M, int64_t K
                                 const uint16_t* bias, uint16_t* y, void* workspace,
                                 size_t ws_bytes, void* stream);
 
+/* Bytes of device workspace ck_linear_w4a8 needs (the same layout and size as the W4A4 linear's). */
+size_t ck_linear_w4a8_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * The W4A8 ConvRot linear, for the "asym_w4a8_int8" packed format of
+ * stable-diffusion.cpp PR #2276 (Summary; read as int4 weights against int8
+ * activations, no weight zero point): every row of x is rotated as in
+ * ck_rotate_quant_rowwise and quantized to INT8 codes (qmax = 127), then
+ * multiplied with the packed int4 weights on the same routes as ck_linear_w4a4
+ * (tensor-core GEMM, or the decode GEMV for M <= 64, K <= 4096,
+ * K % 128 == 0), with the same epilogue:
+ *   y[m,n] = bf16_rne( (float(sum_k q8[m,k] (u[n,k] - 8)) * s_m) * w_scale[n] (+ bias[n]) )
+ * The result equals ck_rotate_quant_rowwise(bits=8) followed by ck_gemm_w4a8
+ * bit for bit. K % 32 == 0 and K % group_size == 0; K <= 1118481 (int32
+ * accumulator).
+ * workspace : at least ck_linear_w4a8_workspace_bytes(M, K) bytes, 256-byte
+ *             aligned, opaque.
+ * Other arguments as for ck_linear_w4a4.
+ */
+ck_status ck_linear_w4a8(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N,
+                         int64_t ldx, int group_size, const uint8_t* w_packed,
+                         const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * ck_linear_w4a4 on weights already unpacked to int8: the weight-cache
+ * trade of comfy-kitchen PR #212 ("[Perf][Ascend] Reuse unpacked W4A4 weights
+ * within an explicit scope", Summary and "Memory and support limits"), where
+ * the caller unpacks the packed weights once (ck_unpack_int4) and reuses the
+ * int8 copy across calls. The int8 copy costs twice the packed bytes of
+ * device memory; in exchange the GEMM loads both operands as int8 tiles and
+ * decodes nothing. The result equals ck_linear_w4a4's bit for bit.
+ * w_s8      : (N, K) int8, values u - 8 in [-8, 7] (the output of
+ *             ck_unpack_int4 on the packed weights), 16-byte aligned.
+ * workspace : at least ck_linear_w4a4_workspace_bytes(M, K) bytes.
+ * Always runs the tensor-core GEMM (no small-batch route): meant for large M,
+ * where the in-kernel weight decode is the cost it removes.
+ * Other arguments as for ck_linear_w4a4.
+ */
+ck_status ck_linear_w4a4_predecoded(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t N,
+                                    int64_t ldx, int group_size, const int8_t* w_s8,
+                                    const uint16_t* w_scale, const uint16_t* bias, uint16_t* y,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
 /* Size of the scratch built into the library for ck_linear_w4a4_static: 32 MiB per device. */
 #define CK_LINEAR_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
 
@@ -253,14 +297,22 @@ ck_status ck_linear_w4a4_scaled(const void* x, ck_dtype xt, int64_t M, int64_t K
  * inside the library, reserved by the CUDA runtime when the library's GPU
  * code is loaded on a device. The call allocates and frees nothing.
  *
+ * Cost to every user of the library: loading the library's GPU code on a
+ * device reserves these 32 MiB there for the life of the process (or of the
+ * device's context), whichever entry points the process calls.
+ *
  * Limits and rules:
  * - The scratch must hold ck_linear_w4a4_workspace_bytes(M, K) bytes, i.e.
  *   about M*K + 8*M. Larger problems (for instance M = 8192, K = 10240) get
  *   CK_ERR_UNSUPPORTED with a message naming the sizes, and nothing runs.
  *   M = 8192, K = 3840 fits.
  * - Set-up: the first call on each device (with that device current) looks up
- *   the scratch's device address and caches it. Make that first call before
- *   starting any stream capture.
+ *   the scratch's device address and caches it with the device's current
+ *   context. Make that first call before starting any stream capture. If the
+ *   context changes (after cudaDeviceReset, say) the next call looks the
+ *   address up again.
+ * - x must live on the current device (CK_ERR_INVALID_ARG otherwise): the
+ *   scratch used is the current device's.
  * - Nothing in the scratch needs to start at zero: every byte the GEMM phase
  *   reads is written earlier in the same call by the quantize phase.
  * - There is one scratch per device, shared by every call on that device.
