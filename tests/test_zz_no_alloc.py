@@ -68,3 +68,37 @@ def test_static_rejects_oversize_and_keeps_working(ck):
     torch.cuda.synchronize()
     assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
     ck.device_error_check()
+
+
+@pytest.mark.gpu
+def test_static_call_allocates_no_device_memory(ck):
+    # the entry point's whole claim: with the output preallocated, a call changes neither
+    # torch's allocator nor the device's free memory (after the first call's set-up)
+    dev = torch.device("cuda:0")
+    d = _inputs(512, 3840, 1024, 15, dev, with_bias=True)
+    out = torch.empty(512, 1024, device=dev, dtype=torch.bfloat16)
+    ck.linear_w4a4_static(d["x"], d["w_packed"], d["w_scale"], 64, bias=d["bias"], out=out)
+    torch.cuda.synchronize()
+    alloc0 = torch.cuda.memory_allocated(dev)
+    free0, _ = torch.cuda.mem_get_info(dev)
+    for _ in range(3):
+        ck.linear_w4a4_static(d["x"], d["w_packed"], d["w_scale"], 64, bias=d["bias"], out=out)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated(dev) == alloc0
+    free1, _ = torch.cuda.mem_get_info(dev)
+    assert free1 == free0
+    ref = ck.linear_w4a4(d["x"], d["w_packed"], d["w_scale"], 64, bias=d["bias"])
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    ck.device_error_check()
+
+
+@pytest.mark.gpu
+def test_static_rejects_input_not_on_the_current_device(ck):
+    # the scratch belongs to the current device, so x must live there: host memory is refused
+    x = torch.zeros(8, 128, dtype=torch.bfloat16)
+    torch.cuda.init()
+    st = ck.lib.ck_linear_w4a4_static(ck._ptr(x), 0, 8, 128, 64, 128, 64, ck._ptr(x), ck._ptr(x), None,
+                                      ck._ptr(x), None)
+    assert st == ck.CK_ERR_INVALID_ARG
+    assert "device" in ck.last_error()
+    ck.device_error_check()
