@@ -21,6 +21,7 @@
 #include "gemv_awq.cuh"
 #include "gemv_stream.cuh"
 #include "gemv_w4a8.cuh"
+#include "gemv_w4a8_stream.cuh"
 #include "gemv_w4a8_tc.cuh"
 #include "rotate_quant.cuh"
 #include "rotate_quant_general.cuh"
@@ -971,6 +972,57 @@ ck_status gemv_w4a8_tc_launch(const int8_t* xq, const float* x_scale, int64_t M,
   return launch_status("gemv_w4a8_tc");
 }
 
+// Tiles the row-split W4A8 kernel fills while the previous kernel still runs, at most
+// this many in flight (see gemv_w4a8_stream.cuh).
+constexpr int kRowsplitFill = 3;
+
+// The row-split W4A8 GEMV (M <= 8, K <= 4096, K % 128 == 0, N % 8 == 0, 16-byte
+// aligned scales and bias). CK_ERR_UNSUPPORTED, with nothing launched, when a
+// CTA's share of rows would leave its ring fewer than two stages.
+ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
+                             const uint8_t* w_packed, const __nv_bfloat16* sw, const __nv_bfloat16* bb,
+                             __nv_bfloat16* yy, cudaStream_t st) {
+  using namespace ck::w4s;
+  const int64_t octets = N / 8;
+  const int grid = (int)std::min<int64_t>(octets, sm_count());
+  Params p;
+  p.xq = xq; p.xs = x_scale; p.sw = sw; p.bias = bb; p.y = yy;
+  p.M = (int)M; p.K = (int)K; p.N = (int)N;
+  p.stage_bytes = (int)((16 * (K / 2) + 1023) / 1024 * 1024);
+  p.max_rows = (int)(8 * ((octets + grid - 1) / grid));
+  p.max_tiles = (p.max_rows + TR - 1) / TR;
+  const int acc_bytes = p.max_tiles * TR * 8 * 4;
+  const int misc_bytes = (64 + 2 * 2 * p.max_rows + 4 + 15) / 16 * 16;
+  const int bar_bytes = (2 * kMaxStages + 1 + p.max_tiles) * 8;
+  const int fixed = acc_bytes + misc_bytes + bar_bytes + 1024;   // 1024: base alignment slack
+  p.ns = std::min(kMaxStages, (kStreamSmemMax - fixed) / p.stage_bytes);
+  if (p.ns < 2 || fixed > kStreamSmemMax) return CK_ERR_UNSUPPORTED;
+  p.fill = kRowsplitFill;
+  p.off_acc = p.ns * p.stage_bytes;
+  p.off_misc = p.off_acc + acc_bytes;
+  p.off_bar = p.off_misc + misc_bytes;
+  const int total = p.off_bar + bar_bytes + 1024;
+  CUtensorMap tw;
+  ck_status r = make_tmap_wtile(&tw, w_packed, (uint64_t)N, (uint64_t)K, TR);
+  if (r != CK_OK) return r;
+  const int cpw = (int)((K / 128 + kCons - 1) / kCons);
+  cudaError_t e;
+#define CK_W4A8_ROWSPLIT(CPW)                                                                      \
+  {                                                                                                \
+    auto kern = w4a8_rowsplit_kernel<CPW>;                                                         \
+    struct Tag {};                                                                                 \
+    e = set_smem_max<Tag>(kern, total);                                                            \
+    if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), total, st, tw, p);      \
+  }
+  if (cpw <= 1) CK_W4A8_ROWSPLIT(1)
+  else if (cpw == 2) CK_W4A8_ROWSPLIT(2)
+  else if (cpw == 3) CK_W4A8_ROWSPLIT(3)
+  else CK_W4A8_ROWSPLIT(4)
+#undef CK_W4A8_ROWSPLIT
+  if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
+  return launch_status("gemv_w4a8");
+}
+
 }  // namespace
 
 extern "C" {
@@ -990,6 +1042,11 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
   const auto* sw = reinterpret_cast<const __nv_bfloat16*>(w_scale);
   const auto* bb = reinterpret_cast<const __nv_bfloat16*>(bias);
   auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
+  if (K <= 4096 && M <= 8 && N % 8 == 0 && aligned(sw, 16) && (bb == nullptr || aligned(bb, 16))) {
+    // row-split streaming path: whole octets of rows per CTA, 16-row tiles (gemv_w4a8_stream.cuh)
+    ck_status r = gemv_w4a8_rowsplit(xq, x_scale, M, K, N, w_packed, sw, bb, yy, S(stream));
+    if (r != CK_ERR_UNSUPPORTED) return r;
+  }
   if (K <= 4096 && M <= 8) {
     // streaming path for up to 8 activation rows: 16-row weight tiles as the m16 operand
     using namespace ck::gstream;

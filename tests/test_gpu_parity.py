@@ -548,6 +548,36 @@ def test_gemv_w4a8_ragged_bit_exact(ck, M, K, N, bias):
     np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
 
 
+@pytest.mark.parametrize("M,K,N,bias", [(1, 128, 8, False), (8, 128, 16, True), (5, 384, 24, True), (2, 4096, 40, False),
+                                        (7, 1024, 1000, True), (4, 2048, 2376, False), (8, 4096, 4736, True),
+                                        (3, 512, 12288, False)])
+def test_gemv_w4a8_rowsplit_shapes_bit_exact(ck, M, K, N, bias):
+    # the row-split streaming kernel (M <= 8, N % 8 == 0): CTAs owning one octet of rows, the last
+    # tile of a CTA moved back over rows an earlier tile wrote, K from one chunk to 32 chunks
+    g = torch.Generator().manual_seed(M * 7919 + N)
+    xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    xs = torch.rand(M, generator=g) * 0.1 + 0.001
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N,), 0.005, 0.02, g)
+    b = WL.uniform((N,), -1, 1, g) if bias else None
+    y = ck.gemv_w4a8(xq.to(DEV), xs.to(DEV), wp.to(DEV), sw.to(DEV), None if b is None else b.to(DEV))
+    r = O.gemv_w4a8(xq.numpy(), xs.numpy(), wp.numpy(), to_np_f64(sw), None if b is None else to_np_f64(b))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
+
+
+def test_gemv_w4a8_unaligned_scales_take_another_path(ck):
+    # scales that are not 16-byte aligned cannot be bulk-copied: the call still gives the exact result
+    M, K, N = 4, 512, 64
+    g = torch.Generator().manual_seed(5)
+    xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    xs = torch.rand(M, generator=g) * 0.1 + 0.001
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    sw = WL.uniform((N + 1,), 0.005, 0.02, g)
+    y = ck.gemv_w4a8(xq.to(DEV), xs.to(DEV), wp.to(DEV), sw.to(DEV)[1:])
+    r = O.gemv_w4a8(xq.numpy(), xs.numpy(), wp.numpy(), to_np_f64(sw[1:]))
+    np.testing.assert_array_equal(bf16_tensor_bits(y), r["y_bits"])
+
+
 def _tall_sample(N, seed):
     rng = np.random.default_rng(seed)
     return np.unique(np.r_[0, 1, 2, N // 2, N - 2, N - 1, rng.integers(0, N, 300)])
