@@ -83,7 +83,7 @@ __device__ __forceinline__ int wtile_addr(int r, int b) {
 }
 
 __device__ __forceinline__ void mma_s8u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 "
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
@@ -146,6 +146,14 @@ __global__ void __launch_bounds__(kThreads, 2) w4a8_stream_kernel(const W4A8Para
     fence_mbarrier_init();
     for (int i = 0; i < min(ns, nt); ++i) issue(i);
   }
+  if (warp == W_EPI) {
+    // this CTA's column scales and biases: constant data, read before the dependency wait
+    const int r0 = 8 * t0, nr = min(8 * nt, p.N - r0);
+    for (int r = lane; r < nr; r += 32) {
+      colv[r] = __bfloat162float(p.sw[r0 + r]);
+      colv[8 * ((p.ntiles + gridDim.x - 1) / gridDim.x) + r] = p.bias ? __bfloat162float(p.bias[r0 + r]) : 0.0f;
+    }
+  }
   grid_dep_launch();
   grid_dep_wait();   // the activations and the output belong to the previous kernel until here
 
@@ -193,13 +201,6 @@ __global__ void __launch_bounds__(kThreads, 2) w4a8_stream_kernel(const W4A8Para
     if (t == 0) {
       xsum_part[warp * 16 + g] = xs_g;
       xsum_part[warp * 16 + g + 8] = xs_g8;
-    }
-  } else if (warp == W_EPI) {
-    // this CTA's column scales and biases
-    const int r0 = 8 * t0, nr = min(8 * nt, p.N - r0);
-    for (int r = lane; r < nr; r += 32) {
-      colv[r] = __bfloat162float(p.sw[r0 + r]);
-      colv[8 * ((p.ntiles + gridDim.x - 1) / gridDim.x) + r] = p.bias ? __bfloat162float(p.bias[r0 + r]) : 0.0f;
     }
   }
   __syncthreads();
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 2) w4a8_stream_kernel(const W4A8Para
 // ============================================== W4A8, at most 8 activation rows
 
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
@@ -536,6 +537,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     fence_mbarrier_init();
     for (int i = 0; i < min(ns, nt); ++i) issue(i);
   }
+  if (warp == W_EPI) {   // bias of this CTA's rows: constant data, read before the dependency wait
+    const int r0 = 16 * t0, nr = min(16 * nt, p.N - r0);
+    for (int r = lane; r < nr; r += 32) colb[r] = p.bias ? Tr::tof(reinterpret_cast<const T*>(p.bias)[r0 + r]) : 0.0f;
+  }
   grid_dep_launch();
   grid_dep_wait();   // the activations and the output belong to the previous kernel until here
 
@@ -566,9 +571,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       X[i][0] = Xc[0];
       X[i][1] = Xc[1];
     }
-  } else if (warp == W_EPI) {
-    const int r0 = 16 * t0, nr = min(16 * nt, p.N - r0);
-    for (int r = lane; r < nr; r += 32) colb[r] = p.bias ? Tr::tof(reinterpret_cast<const T*>(p.bias)[r0 + r]) : 0.0f;
   }
   __syncthreads();
   volatile int* abort = abort_flag;

@@ -28,6 +28,15 @@
  * - Kernels that wait on shared-memory barriers give up after a bounded time
  *   and set a device error word instead of hanging; ck_device_error_check()
  *   reports it.
+ * - Back-to-back calls overlap: every kernel is launched as a programmatic
+ *   dependent of the previous kernel on the stream and waits for it before it
+ *   reads activations or writes outputs. The decode GEMVs (and the linears'
+ *   small-batch route, which runs them) treat their WEIGHT operands --
+ *   packed weights, weight scales, zeros and bias -- as constant data and
+ *   start streaming them before that wait. So do not let the kernel launched
+ *   immediately before such a call on the same stream write those weights;
+ *   any other operation in between (another kernel, a copy, an event wait)
+ *   makes the ordering complete again.
  */
 #ifndef CK_H_
 #define CK_H_
