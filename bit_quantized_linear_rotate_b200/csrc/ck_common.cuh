@@ -68,23 +68,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-#ifdef CK_WAIT_HINT_NS
-// try_wait that lets the hardware suspend the thread until the phase completes
-// (or up to the hint): a waiting warp then takes no issue slots from the warps
-// that compute.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "n"(CK_WAIT_HINT_NS)
-      : "memory");
-  return ok != 0;
-}
-#endif
-
 // Waits until the phase with the given parity has completed. Gives up after
 // `limit_ns` (or at once if *abort is already set), records the timeout in the
 // device error word and in *abort, and returns false. Never spins forever.
@@ -93,17 +76,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           uint64_t limit_ns = kDefaultWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
-#ifdef CK_WAIT_HINT_NS
-  for (;;) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
-    if (abort != nullptr && *abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      if (abort != nullptr) *abort = 1;
-      report_timeout(site);
-      return false;
-    }
-  }
-#else
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0u) {
@@ -115,7 +87,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
-#endif
 }
 
 // Cluster-scope variants, for barriers that receive arrivals from the peer CTA
