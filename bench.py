@@ -398,7 +398,7 @@ def time_gemvs(ck, dev, hbm_gbs: float, iters: int = 200):
         out[f"w4a8_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,
                              "all_GBps": allb / (ms * 1e-3) / 1e9,
                              "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / hbm_gbs, "copies": R,
-                             "traffic": load_traffic("w4a8_rowsplit_kernel" if M <= 8 else "w4a8_stream_kernel")}
+                             "traffic": load_traffic("w4a8_rowsplit_kernel" if M <= 8 else "w4a8_rowsplit_kernel_m16")}
         # the same product on the tcgen05 alternative (not the default path)
         ms = time_rotating(lambda c: ck.gemv_w4a8_tc(xq, xs, wps[c], sw, out=y), R, iters, 10)
         out[f"w4a8_tc_M{M}"] = {"us": ms * 1e3, "weight_GBps": wbytes / (ms * 1e-3) / 1e9,

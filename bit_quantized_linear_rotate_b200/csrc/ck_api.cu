@@ -151,17 +151,18 @@ int current_device() {
   return dev;
 }
 
-// Raises a stream kernel's dynamic shared-memory limit to kStreamSmemMax (the
-// most any of its launches asks for, `bytes` <= kStreamSmemMax) once per
-// device, cached per kernel instantiation through Tag.
+// Raises a stream kernel's dynamic shared-memory limit to max_bytes (the most
+// any of its launches asks for, `bytes` <= max_bytes; kStreamSmemMax unless the
+// kernel runs one CTA per SM) once per device, cached per kernel instantiation
+// through Tag.
 template <typename Tag, typename KernelT>
-cudaError_t set_smem_max(KernelT kern, int bytes) {
+cudaError_t set_smem_max(KernelT kern, int bytes, int max_bytes = kStreamSmemMax) {
   static std::atomic<bool> done[kMaxDevices];
   const int dev = current_device();
   if (dev < 0) return cudaErrorInvalidDevice;
-  if (bytes > kStreamSmemMax) return cudaErrorInvalidValue;
+  if (bytes > max_bytes) return cudaErrorInvalidValue;
   if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
   if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
   return e;
 }
@@ -466,7 +467,12 @@ size_t linear_ws_bytes(int64_t M, int64_t K) {
 // same, so the results do not depend on the route. Both phases of the linear
 // take the decision from (M, K) alone.
 bool linear_small_m(int64_t M, int64_t K) { return M <= 64 && K % 128 == 0 && K <= 4096; }
-constexpr int64_t kSmallMChunk = 16;   // rows per GEMV call
+constexpr int64_t kSmallMChunk = 16;           // rows per GEMV call
+constexpr int64_t kSmallMChunkRowsplit = 32;   // rows per row-split GEMV call
+
+ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
+                             const uint8_t* w_packed, const __nv_bfloat16* sw, const __nv_bfloat16* bb,
+                             __nv_bfloat16* yy, cudaStream_t st);
 
 ck_status check_linear_workspace(const char* who, int64_t M, int64_t K, const void* ws, size_t bytes) {
   if (ws == nullptr || bytes < linear_ws_bytes(M, K))
@@ -700,9 +706,23 @@ ck_status linear_matmul_entry(const char* who, int64_t M, int64_t K, int64_t N, 
     return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
   LinearWs ws = linear_ws(const_cast<void*>(workspace), M, K);
   if (linear_small_m(M, K)) {
-    for (int64_t r0 = 0; r0 < M; r0 += kSmallMChunk) {
-      const int64_t mc = std::min<int64_t>(kSmallMChunk, M - r0);
-      r = ck_gemv_w4a8(ws.q + r0 * K, ws.scale + r0, mc, K, N, w_packed, w_scale, bias, y + r0 * N, stream);
+    // 32-row pieces through the row-split kernel where it applies, else 16-row GEMV calls
+    const bool rowsplit = N % 8 == 0 && aligned(w_scale, 16) && (bias == nullptr || aligned(bias, 16));
+    for (int64_t r0 = 0; r0 < M; r0 += kSmallMChunkRowsplit) {
+      const int64_t mc = std::min<int64_t>(kSmallMChunkRowsplit, M - r0);
+      r = CK_ERR_UNSUPPORTED;
+      if (rowsplit)
+        r = gemv_w4a8_rowsplit(ws.q + r0 * K, ws.scale + r0, mc, K, N, w_packed,
+                               reinterpret_cast<const __nv_bfloat16*>(w_scale),
+                               reinterpret_cast<const __nv_bfloat16*>(bias),
+                               reinterpret_cast<__nv_bfloat16*>(y + r0 * N), S(stream));
+      if (r == CK_ERR_UNSUPPORTED) {   // nothing launched: 16-row GEMV calls
+        for (int64_t q0 = r0; q0 < r0 + mc; q0 += kSmallMChunk) {
+          const int64_t qc = std::min<int64_t>(kSmallMChunk, r0 + mc - q0);
+          r = ck_gemv_w4a8(ws.q + q0 * K, ws.scale + q0, qc, K, N, w_packed, w_scale, bias, y + q0 * N, stream);
+          if (r != CK_OK) return r;
+        }
+      }
       if (r != CK_OK) return r;
     }
     return ok();
@@ -975,14 +995,21 @@ ck_status gemv_w4a8_tc_launch(const int8_t* xq, const float* x_scale, int64_t M,
 // Tiles the row-split W4A8 kernel fills while the previous kernel still runs, at most
 // this many in flight (see gemv_w4a8_stream.cuh).
 constexpr int kRowsplitFill = 3;
+// Dynamic shared memory of a row-split CTA for more than 8 tokens: one CTA per SM
+// (the 228 KB of an SM less the 1 KB the runtime reserves per CTA).
+constexpr int kRowsplitSmemBig = 227 * 1024;
 
-// The row-split W4A8 GEMV (M <= 8, K <= 4096, K % 128 == 0, N % 8 == 0, 16-byte
+// The row-split W4A8 GEMV (M <= 32, K <= 4096, K % 128 == 0, N % 8 == 0, 16-byte
 // aligned scales and bias). CK_ERR_UNSUPPORTED, with nothing launched, when a
 // CTA's share of rows would leave its ring fewer than two stages.
 ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
                              const uint8_t* w_packed, const __nv_bfloat16* sw, const __nv_bfloat16* bb,
                              __nv_bfloat16* yy, cudaStream_t st) {
   using namespace ck::w4s;
+  if (M > kMaxTokens || K > 4096 || K % 128 != 0 || N % 8 != 0) return CK_ERR_UNSUPPORTED;
+  const int nt = M <= 8 ? 1 : M <= 16 ? 2 : 4;
+  const int ncons = cons_warps(nt), nthreads = threads_for(nt);
+  const int smax = nt == 1 ? kStreamSmemMax : kRowsplitSmemBig;
   const int64_t octets = N / 8;
   const int grid = (int)std::min<int64_t>(octets, sm_count());
   Params p;
@@ -991,12 +1018,16 @@ ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, 
   p.stage_bytes = (int)((16 * (K / 2) + 1023) / 1024 * 1024);
   p.max_rows = (int)(8 * ((octets + grid - 1) / grid));
   p.max_tiles = (p.max_rows + TR - 1) / TR;
-  const int acc_bytes = p.max_tiles * TR * 8 * 4;
-  const int misc_bytes = (64 + 2 * 2 * p.max_rows + 4 + 15) / 16 * 16;
+  const int acc_bytes = p.max_tiles * nt * 8 * TS * 4;
+  const int misc_bytes = (2 * kMaxTokens * 4 + 2 * 2 * p.max_rows + 4 + 15) / 16 * 16;
   const int bar_bytes = (2 * kMaxStages + 1 + p.max_tiles) * 8;
   const int fixed = acc_bytes + misc_bytes + bar_bytes + 1024;   // 1024: base alignment slack
-  p.ns = std::min(kMaxStages, (kStreamSmemMax - fixed) / p.stage_bytes);
-  if (p.ns < 2 || fixed > kStreamSmemMax) return CK_ERR_UNSUPPORTED;
+  if (fixed > smax) return CK_ERR_UNSUPPORTED;
+  p.ns = std::min(kMaxStages, (smax - fixed) / p.stage_bytes);
+  if (p.ns < 2) return CK_ERR_UNSUPPORTED;
+  // no more stages than a CTA has tiles: the shared memory left over lets the neighbouring
+  // kernels' CTAs stay resident beside this one
+  p.ns = std::min(p.ns, std::max(2, p.max_tiles));
   p.fill = kRowsplitFill;
   p.off_acc = p.ns * p.stage_bytes;
   p.off_misc = p.off_acc + acc_bytes;
@@ -1005,19 +1036,27 @@ ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, 
   CUtensorMap tw;
   ck_status r = make_tmap_wtile(&tw, w_packed, (uint64_t)N, (uint64_t)K, TR);
   if (r != CK_OK) return r;
-  const int cpw = (int)((K / 128 + kCons - 1) / kCons);
-  cudaError_t e;
-#define CK_W4A8_ROWSPLIT(CPW)                                                                      \
+  const int cpw = (int)((K / 128 + ncons - 1) / ncons);
+  cudaError_t e = cudaSuccess;
+#define CK_W4A8_ROWSPLIT(NT, CPW)                                                                  \
   {                                                                                                \
-    auto kern = w4a8_rowsplit_kernel<CPW>;                                                         \
+    auto kern = w4a8_rowsplit_kernel<NT, CPW>;                                                     \
     struct Tag {};                                                                                 \
-    e = set_smem_max<Tag>(kern, total);                                                            \
-    if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(kThreads), total, st, tw, p);      \
+    e = set_smem_max<Tag>(kern, total, smax);                                                      \
+    if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(nthreads), total, st, tw, p);      \
   }
-  if (cpw <= 1) CK_W4A8_ROWSPLIT(1)
-  else if (cpw == 2) CK_W4A8_ROWSPLIT(2)
-  else if (cpw == 3) CK_W4A8_ROWSPLIT(3)
-  else CK_W4A8_ROWSPLIT(4)
+  if (nt == 1) {
+    if (cpw <= 1) CK_W4A8_ROWSPLIT(1, 1)
+    else if (cpw == 2) CK_W4A8_ROWSPLIT(1, 2)
+    else if (cpw == 3) CK_W4A8_ROWSPLIT(1, 3)
+    else CK_W4A8_ROWSPLIT(1, 4)
+  } else if (nt == 2) {
+    if (cpw <= 1) CK_W4A8_ROWSPLIT(2, 1)
+    else CK_W4A8_ROWSPLIT(2, 2)
+  } else {
+    if (cpw <= 1) CK_W4A8_ROWSPLIT(4, 1)
+    else CK_W4A8_ROWSPLIT(4, 2)
+  }
 #undef CK_W4A8_ROWSPLIT
   if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
   return launch_status("gemv_w4a8");
@@ -1042,7 +1081,7 @@ ck_status ck_gemv_w4a8(const int8_t* xq, const float* x_scale, int64_t M, int64_
   const auto* sw = reinterpret_cast<const __nv_bfloat16*>(w_scale);
   const auto* bb = reinterpret_cast<const __nv_bfloat16*>(bias);
   auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
-  if (K <= 4096 && M <= 8 && N % 8 == 0 && aligned(sw, 16) && (bb == nullptr || aligned(bb, 16))) {
+  if (K <= 4096 && N % 8 == 0 && aligned(sw, 16) && (bb == nullptr || aligned(bb, 16))) {
     // row-split streaming path: whole octets of rows per CTA, 16-row tiles (gemv_w4a8_stream.cuh)
     ck_status r = gemv_w4a8_rowsplit(xq, x_scale, M, K, N, w_packed, sw, bb, yy, S(stream));
     if (r != CK_ERR_UNSUPPORTED) return r;

@@ -9,6 +9,7 @@ Cases (full workload sizes, a few GB at most on the device):
   gemm_s8_M8192    ck_gemm_s8 with pre-decoded int8 weights
   gemm_w4a4_M8192  ck_gemm_w4a4, packed int4 activations and weights
   linear_M8192     ck_linear_w4a4 (both kernels)
+  linear_M32       ck_linear_w4a4 at M=32, K=N=3840 (the small-batch route)
   linmm_M8192      ck_linear_w4a4_matmul (the linear's GEMM phase alone)
   linq_M8192       ck_linear_w4a4_quantize (the linear's rotate + quantize phase alone)
   w4a8_M{1,4,16}   ck_gemv_w4a8, K=4096, N=12288
@@ -30,7 +31,7 @@ from . import workloads as WL
 
 def build_case(name: str, dev):
     if name.startswith(("rq_", "gemm_", "lin")):
-        w = WL.LINEAR_M8192
+        w = WL.LINEAR_M32 if name == "linear_M32" else WL.LINEAR_M8192
         if name == "rq_M8192_K10240_G16":
             x = WL.linear_inputs(WL.LINEAR_MLP_DOWN)["x"].to(dev)
             return lambda: ck.rotate_quant_rowwise(x, 16, 8)
@@ -50,7 +51,7 @@ def build_case(name: str, dev):
             qp, _ = ck.rotate_quant_rowwise(x, w.G, 4)
             return lambda: ck.gemm_w4a4(qp, sa, wp, sw, out=y)
         ws = torch.empty(ck.linear_w4a4_workspace_bytes(w.M, w.K), device=dev, dtype=torch.uint8)
-        if name == "linear_M8192":
+        if name in ("linear_M8192", "linear_M32"):
             return lambda: ck.linear_w4a4(x, wp, sw, w.G, workspace=ws, out=y)
         if name == "linq_M8192":
             return lambda: ck.linear_w4a4_quantize(x, w.G, ws)

@@ -373,7 +373,8 @@ def _linear_workspace(ws, M, K):
 
 
 @pytest.mark.parametrize("M,K,N", [(300, 1024, 520), (32, 3840, 520), (1, 1024, 96), (64, 1024, 520),
-                                   (65, 1024, 520), (17, 128, 72)])
+                                   (65, 1024, 520), (17, 128, 72), (24, 2048, 1000), (40, 512, 264),
+                                   (33, 256, 100), (32, 4096, 4736)])
 def test_linear_phases_equal_rotate_quant_plus_gemm_w4a4(ck, M, K, N):
     # both routes of the linear (tensor-core GEMM; decode GEMV for small batches) give the
     # result of rotate_quant(bits = 4) followed by the packed-activation GEMM, bit for bit
@@ -550,10 +551,12 @@ def test_gemv_w4a8_ragged_bit_exact(ck, M, K, N, bias):
 
 @pytest.mark.parametrize("M,K,N,bias", [(1, 128, 8, False), (8, 128, 16, True), (5, 384, 24, True), (2, 4096, 40, False),
                                         (7, 1024, 1000, True), (4, 2048, 2376, False), (8, 4096, 4736, True),
-                                        (3, 512, 12288, False)])
+                                        (3, 512, 12288, False), (9, 128, 8, True), (12, 384, 24, False),
+                                        (16, 4096, 4736, True), (13, 3840, 3840, False), (16, 2048, 12288, True)])
 def test_gemv_w4a8_rowsplit_shapes_bit_exact(ck, M, K, N, bias):
-    # the row-split streaming kernel (M <= 8, N % 8 == 0): CTAs owning one octet of rows, the last
-    # tile of a CTA moved back over rows an earlier tile wrote, K from one chunk to 32 chunks
+    # the row-split streaming kernel (M <= 16, N % 8 == 0; one token group up to M = 8, two
+    # above): CTAs owning one octet of rows, the last tile of a CTA moved back over rows an
+    # earlier tile wrote, K from one chunk to 32 chunks
     g = torch.Generator().manual_seed(M * 7919 + N)
     xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
     xs = torch.rand(M, generator=g) * 0.1 + 0.001
