@@ -71,6 +71,12 @@ struct Params {
   int off_acc, off_misc, off_bar; // shared-memory offsets
 };
 
+// The consumer warps' named barrier (id 1; __syncthreads takes id 0).
+template <int NC>
+__device__ __forceinline__ void cons_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
+}
+
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
@@ -213,9 +219,21 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
 
       // row g of chunk c sits at line (c * 16 + g) of the swizzled tile; row g + 8 eight lines on
       const int wb = (warp * 16 + g) * 64 + ((t ^ ((g >> 1) & 3)) << 4);
+      // With consumer-written outputs the consumer warps meet at a named barrier once per tile;
+      // after a timeout a warp skips the work but still takes every barrier, so that all of
+      // them reach the same count (every other wait is bounded).
+      bool ok = true;
       for (int i = 0; i < ntile; ++i) {
         const int s = i % ns;
-        if (!warp_wait(&full[s], (i / ns) & 1, abort, 30)) break;
+        if constexpr (kConsEpi) {
+          ok = ok && warp_wait(&full[s], (i / ns) & 1, abort, 30);
+          if (!ok) {
+            cons_bar_sync<NC>();
+            continue;
+          }
+        } else {
+          if (!warp_wait(&full[s], (i / ns) & 1, abort, 30)) break;
+        }
         const uint8_t* st = sm + s * p.stage_bytes;
         // with four token groups the activation fragments fill most registers: the weight words
         // of a chunk are read just before its MMAs and the stage is handed back after the last
@@ -262,11 +280,11 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
               } else {
                 const uint32_t hi[4] = {(u[2 * pr] >> 4) & 0x0F0F0F0Fu, (v[2 * pr] >> 4) & 0x0F0F0F0Fu,
                                         (u[2 * pr + 1] >> 4) & 0x0F0F0F0Fu, (v[2 * pr + 1] >> 4) & 0x0F0F0F0Fu};
+                // the groups' MMAs interleave, so that two on one accumulator are NT apart
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                  mma_u8s8(alo[nt], lo, bf[ci][2 * pr][0][nt], bf[ci][2 * pr + 1][0][nt]);
-                  mma_u8s8(alo[nt], hi, bf[ci][2 * pr][1][nt], bf[ci][2 * pr + 1][1][nt]);
-                }
+                for (int nt = 0; nt < NT; ++nt) mma_u8s8(alo[nt], lo, bf[ci][2 * pr][0][nt], bf[ci][2 * pr + 1][0][nt]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_u8s8(alo[nt], hi, bf[ci][2 * pr][1][nt], bf[ci][2 * pr + 1][1][nt]);
               }
             }
           }
@@ -290,13 +308,15 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
           atomicAdd(so + 8, alo[nt][2]);
           atomicAdd(so + TS + 8, alo[nt][3]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tdone[i]);   // release: the adds above reach the epilogue
-        if constexpr (kConsEpi) {
+        if constexpr (!kConsEpi) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tdone[i]);   // release: the adds above reach the epilogue
+        } else {
           // once every consumer warp has added its part, output o = 32 warp + lane of the
           // tile's 16 x 8 NT: token o / 16, row o % 16 (a half warp stores 16 adjacent rows)
-          if (i == 0 && !warp_wait(cbar, 0, abort, 36)) break;
-          if (!warp_wait(&tdone[i], 0, abort, 34)) break;
+          if (i == 0) ok = warp_wait(cbar, 0, abort, 36);
+          cons_bar_sync<NC>();
+          if (!ok) continue;
           const int o = warp * 32 + lane;
           const int tk = o >> 4, r = o & 15;
           const int ts = tstart(i);
