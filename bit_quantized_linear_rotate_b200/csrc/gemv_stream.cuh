@@ -22,12 +22,13 @@
 //
 // Back-to-back calls overlap: a CTA takes at most half of an SM's shared
 // memory, the kernels are launched as programmatic dependents, each lets the
-// next one be scheduled as soon as it starts, and a new call streams its first
-// weight tiles (constant data) into its ring while the previous call is still
-// running; only the activation reads and the output writes wait for the
-// previous kernel (grid_dep_wait). A decode loop of GEMVs thus keeps HBM
-// streaming across kernel boundaries instead of paying each launch's ramp-up
-// and drain.
+// next one be scheduled once its consumers have their activations (trigger
+// note: a next call's weight prefetch would otherwise queue ahead of those
+// loads), and a new call streams its first weight tiles (constant data) into
+// its ring while the previous call is still running; only the activation
+// reads and the output writes wait for the previous kernel (grid_dep_wait).
+// A decode loop of GEMVs thus keeps HBM streaming across kernel boundaries
+// instead of paying each launch's ramp-up and drain.
 //
 // W4A8 (comfy-kitchen PR #182, "Description": register-side int4 decode, int32
 // accumulation, EpiRowwise): weights are the n8 operand of
@@ -154,7 +155,6 @@ __global__ void __launch_bounds__(kThreads, 2) w4a8_stream_kernel(const W4A8Para
       colv[8 * ((p.ntiles + gridDim.x - 1) / gridDim.x) + r] = p.bias ? __bfloat162float(p.bias[r0 + r]) : 0.0f;
     }
   }
-  grid_dep_launch();
   grid_dep_wait();   // the activations and the output belong to the previous kernel until here
 
   uint32_t af[CPW][4][4];
@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 2) w4a8_stream_kernel(const W4A8Para
     }
   }
   __syncthreads();
+  grid_dep_launch();   // once every consumer has its activations (the trigger note above)
   volatile int* abort = abort_flag;
 
   if (warp < kCons) {
@@ -344,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     fence_mbarrier_init();
     for (int i = 0; i < min(ns, nt); ++i) issue(i);
   }
-  grid_dep_launch();
   grid_dep_wait();   // the activations and the output belong to the previous kernel until here
 
   uint32_t bf[CPW][4][2];   // activation fragments of token g
@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   __syncthreads();
+  grid_dep_launch();   // once every consumer has its activations (the trigger note above)
   volatile int* abort = abort_flag;
 
   if (warp < kCons) {
@@ -541,7 +542,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int r0 = 16 * t0, nr = min(16 * nt, p.N - r0);
     for (int r = lane; r < nr; r += 32) colb[r] = p.bias ? Tr::tof(reinterpret_cast<const T*>(p.bias)[r0 + r]) : 0.0f;
   }
-  grid_dep_launch();
   grid_dep_wait();   // the activations and the output belong to the previous kernel until here
 
   uint32_t bp[SPW][8];    // activation fragments (token g, k = sb*64 + 16t + (k, k+4) pairs)
@@ -573,6 +573,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   __syncthreads();
+  grid_dep_launch();   // once every consumer has its activations (the trigger note above)
   volatile int* abort = abort_flag;
 
   if (warp < kCons) {

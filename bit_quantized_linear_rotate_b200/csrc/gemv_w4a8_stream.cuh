@@ -26,6 +26,11 @@
 //   time, so that the activation loads made after the dependency wait do not
 //   queue behind a whole ring of weight tiles. The weight scales and bias of
 //   the CTA's rows come by bulk copy on their own barrier.
+// * Dependent launch. The next kernel on the stream is released only once
+//   every consumer warp of the CTA has its activation fragments and has
+//   finished the first tile: a next call's weight prefetch would otherwise
+//   queue ahead of this call's activation loads (measured: 6.8 -> 6.3 us a
+//   call at M = 1..4, K = 4096, N = 12288).
 // * Compute. NC consumer warps split K (8 for one token group, 16 and one CTA
 //   per SM for more); each holds its activation fragments in registers. A packed word costs two logical ops: the low nibbles (even k)
 //   and the high nibbles left in place (16 x odd-k value) go to two MMAs with
@@ -148,7 +153,6 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
   for (int i = threadIdx.x; i < ntile * SLOT; i += blockDim.x) acc_sl[i] = 0;
   if (threadIdx.x < kMaxTokens) xsum[threadIdx.x] = 0;
   __syncthreads();
-  grid_dep_launch();
   volatile int* abort = abort_flag;
 
   if (warp == W_PROD) {
@@ -317,6 +321,7 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
           if (i == 0) ok = warp_wait(cbar, 0, abort, 36);
           cons_bar_sync<NC>();
           if (!ok) continue;
+          if (i == 0) grid_dep_launch();   // every consumer warp is past its activation loads
           const int o = warp * 32 + lane;
           const int tk = o >> 4, r = o & 15;
           const int ts = tstart(i);
@@ -343,6 +348,7 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
       float xsc[TPL];
       for (int i = 0; cols_ok && i < ntile; ++i) {
         if (!warp_wait(&tdone[i], 0, abort, 34)) break;
+        if (i == 0) grid_dep_launch();   // every consumer warp is past its activation loads
         if (i == 0) {
 #pragma unroll
           for (int q = 0; q < TPL; ++q) {
