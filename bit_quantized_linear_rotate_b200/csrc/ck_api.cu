@@ -436,12 +436,23 @@ ck_status gemm_impl(const void* qa, int64_t M, int64_t K, int64_t N, const void*
 }
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
-size_t linear_q_bytes(int64_t M, int64_t K) { return align256((size_t)M * (size_t)K); }
+bool linear_small_m(int64_t M, int64_t K);
 
-// The linear's workspace: int8 codes (M, K) in the GEMM's permuted column order,
-// float32 row scales (M), int32 row sums of the codes (M), each 256-byte aligned.
+// The codes' region of the linear's workspace. Small batches: the codes packed two
+// per byte, then room for them one per byte (used only when the matmul phase must
+// take a GEMV path that reads int8).
+size_t linear_q_bytes(int64_t M, int64_t K) {
+  if (linear_small_m(M, K)) return align256((size_t)M * (size_t)K / 2) + align256((size_t)M * (size_t)K);
+  return align256((size_t)M * (size_t)K);
+}
+
+// The linear's workspace: the codes (int8 (M, K) in the GEMM's permuted column
+// order; for small batches packed int4 or, in the W4A8 linear, int8 in natural
+// order), float32 row scales (M), int32 row sums of the codes (M), each 256-byte
+// aligned.
 struct LinearWs {
   int8_t* q;
+  int8_t* q8;   // small batches: room for the packed codes unpacked to int8
   float* scale;
   int32_t* rowsum;
 };
@@ -450,6 +461,7 @@ LinearWs linear_ws(void* base, int64_t M, int64_t K) {
   uint8_t* b = reinterpret_cast<uint8_t*>(base);
   LinearWs w;
   w.q = reinterpret_cast<int8_t*>(b);
+  w.q8 = linear_small_m(M, K) ? reinterpret_cast<int8_t*>(b + align256((size_t)M * (size_t)K / 2)) : nullptr;
   w.scale = reinterpret_cast<float*>(b + linear_q_bytes(M, K));
   w.rowsum = reinterpret_cast<int32_t*>(b + linear_q_bytes(M, K) + align256((size_t)M * sizeof(float)));
   return w;
@@ -467,12 +479,20 @@ size_t linear_ws_bytes(int64_t M, int64_t K) {
 // same, so the results do not depend on the route. Both phases of the linear
 // take the decision from (M, K) alone.
 bool linear_small_m(int64_t M, int64_t K) { return M <= 64 && K % 128 == 0 && K <= 4096; }
+
+// What phase 1 of a linear stores: the GEMM's permuted int8 codes with row sums, or
+// for small batches the codes in natural order, packed two per byte when they are
+// int4 (the row-split GEMV then pulls half the bytes from L2).
+int linear_store(int64_t M, int64_t K, int bits) {
+  if (!linear_small_m(M, K)) return ck::rq::STORE_INT8_PERM;
+  return bits == 4 ? ck::rq::STORE_PACKED4 : ck::rq::STORE_INT8;
+}
 constexpr int64_t kSmallMChunk = 16;           // rows per GEMV call
 constexpr int64_t kSmallMChunkRowsplit = 32;   // rows per row-split GEMV call
 
 ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
                              const uint8_t* w_packed, const __nv_bfloat16* sw, const __nv_bfloat16* bb,
-                             __nv_bfloat16* yy, cudaStream_t st);
+                             __nv_bfloat16* yy, cudaStream_t st, bool a4 = false);
 
 ck_status check_linear_workspace(const char* who, int64_t M, int64_t K, const void* ws, size_t bytes) {
   if (ws == nullptr || bytes < linear_ws_bytes(M, K))
@@ -673,7 +693,7 @@ int64_t linear_term(int bits) { return bits == 4 ? kTermLinear : kTermGemv; }
 // tensor-core GEMM with unsigned weight decode); otherwise the codes stay in
 // natural order (the decode-GEMV route and the pre-decoded-weight GEMM).
 ck_status linear_quantize_entry(const char* who, const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx,
-                                int group_size, int bits, float in_scale, bool perm, void* workspace,
+                                int group_size, int bits, float in_scale, int store, void* workspace,
                                 size_t ws_bytes, void* stream) {
   ck_status r = check_gemm_shape(who, M, K, 1, linear_term(bits));
   if (r != CK_OK) return r;
@@ -687,7 +707,6 @@ ck_status linear_quantize_entry(const char* who, const void* x, ck_dtype xt, int
   if (x == nullptr) return fail(CK_ERR_INVALID_ARG, "%s: null pointer", who);
   if (!aligned(x, 16) || ldx % 8 != 0) return fail(CK_ERR_INVALID_ARG, "%s: x rows must be 16-byte aligned", who);
   LinearWs ws = linear_ws(workspace, M, K);
-  const int store = perm ? ck::rq::STORE_INT8_PERM : ck::rq::STORE_INT8;
   return rotate_quant_impl(x, xt, M, K, ldx, group_size, bits, store, ws.q, ws.scale, ws.rowsum, S(stream),
                            in_scale);
 }
@@ -706,20 +725,29 @@ ck_status linear_matmul_entry(const char* who, int64_t M, int64_t K, int64_t N, 
     return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
   LinearWs ws = linear_ws(const_cast<void*>(workspace), M, K);
   if (linear_small_m(M, K)) {
-    // 32-row pieces through the row-split kernel where it applies, else 16-row GEMV calls
+    // 32-row pieces through the row-split kernel where it applies (int4 codes read packed),
+    // else 16-row GEMV calls on int8 codes (unpacked first when phase 1 packed them)
+    const bool a4 = bits == 4;
     const bool rowsplit = N % 8 == 0 && aligned(w_scale, 16) && (bias == nullptr || aligned(bias, 16));
+    const int8_t* q8 = ws.q;
+    bool unpacked = false;
     for (int64_t r0 = 0; r0 < M; r0 += kSmallMChunkRowsplit) {
       const int64_t mc = std::min<int64_t>(kSmallMChunkRowsplit, M - r0);
       r = CK_ERR_UNSUPPORTED;
       if (rowsplit)
-        r = gemv_w4a8_rowsplit(ws.q + r0 * K, ws.scale + r0, mc, K, N, w_packed,
+        r = gemv_w4a8_rowsplit(a4 ? ws.q + r0 * (K / 2) : ws.q + r0 * K, ws.scale + r0, mc, K, N, w_packed,
                                reinterpret_cast<const __nv_bfloat16*>(w_scale),
                                reinterpret_cast<const __nv_bfloat16*>(bias),
-                               reinterpret_cast<__nv_bfloat16*>(y + r0 * N), S(stream));
+                               reinterpret_cast<__nv_bfloat16*>(y + r0 * N), S(stream), a4);
       if (r == CK_ERR_UNSUPPORTED) {   // nothing launched: 16-row GEMV calls
+        if (a4 && !unpacked) {
+          if ((r = ck_unpack_int4(reinterpret_cast<const uint8_t*>(ws.q), M, K, ws.q8, stream)) != CK_OK) return r;
+          q8 = ws.q8;
+          unpacked = true;
+        }
         for (int64_t q0 = r0; q0 < r0 + mc; q0 += kSmallMChunk) {
           const int64_t qc = std::min<int64_t>(kSmallMChunk, r0 + mc - q0);
-          r = ck_gemv_w4a8(ws.q + q0 * K, ws.scale + q0, qc, K, N, w_packed, w_scale, bias, y + q0 * N, stream);
+          r = ck_gemv_w4a8(q8 + q0 * K, ws.scale + q0, qc, K, N, w_packed, w_scale, bias, y + q0 * N, stream);
           if (r != CK_OK) return r;
         }
       }
@@ -738,7 +766,7 @@ extern "C" {
 ck_status ck_linear_w4a4_quantize(const void* x, ck_dtype xt, int64_t M, int64_t K, int64_t ldx, int group_size,
                                   void* workspace, size_t ws_bytes, void* stream) {
   return linear_quantize_entry("linear_w4a4_quantize", x, xt, M, K, ldx, group_size, 4, 1.0f,
-                               !linear_small_m(M, K), workspace, ws_bytes, stream);
+                               linear_store(M, K, 4), workspace, ws_bytes, stream);
 }
 
 ck_status ck_linear_w4a4_matmul(int64_t M, int64_t K, int64_t N, const uint8_t* w_packed, const uint16_t* w_scale,
@@ -763,7 +791,7 @@ ck_status linear_entry(const char* who, const void* x, ck_dtype xt, int64_t M, i
   if (!aligned(w_packed, 16)) return fail(CK_ERR_UNSUPPORTED, "%s: weights must be 16-byte aligned", who);
   if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
-  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, bits, in_scale, !linear_small_m(M, K), workspace,
+  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, bits, in_scale, linear_store(M, K, bits), workspace,
                             ws_bytes, stream);
   if (r != CK_OK) return r;
   return linear_matmul_entry(who, M, K, N, bits, w_packed, w_scale, bias, y, workspace, ws_bytes, stream);
@@ -811,7 +839,8 @@ ck_status ck_linear_w4a4_predecoded(const void* x, ck_dtype xt, int64_t M, int64
   if (!aligned(w_s8, 16)) return fail(CK_ERR_UNSUPPORTED, "%s: weights must be 16-byte aligned", who);
   if (!aligned(w_scale, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)))
     return fail(CK_ERR_INVALID_ARG, "%s: misaligned scale, bias or output", who);
-  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, 4, 1.0f, false, workspace, ws_bytes, stream);
+  r = linear_quantize_entry(who, x, xt, M, K, ldx, group_size, 4, 1.0f, ck::rq::STORE_INT8, workspace, ws_bytes,
+                            stream);
   if (r != CK_OK) return r;
   LinearWs ws = linear_ws(workspace, M, K);
   return gemm_impl<ck::gemm::OP_INT8, ck::gemm::OP_INT8, ck::gemm::EPI_BF16>(
@@ -1007,7 +1036,7 @@ constexpr int kRowsplitSmemBig = 227 * 1024;
 // CTA's share of rows would leave its ring fewer than two stages.
 ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, int64_t K, int64_t N,
                              const uint8_t* w_packed, const __nv_bfloat16* sw, const __nv_bfloat16* bb,
-                             __nv_bfloat16* yy, cudaStream_t st) {
+                             __nv_bfloat16* yy, cudaStream_t st, bool a4) {
   using namespace ck::w4s;
   if (M > kMaxTokens || K > 4096 || K % 128 != 0 || N % 8 != 0) return CK_ERR_UNSUPPORTED;
   const int nt = M <= 8 ? 1 : M <= 16 ? 2 : 4;
@@ -1041,12 +1070,17 @@ ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, 
   if (r != CK_OK) return r;
   const int cpw = (int)((K / 128 + ncons - 1) / ncons);
   cudaError_t e = cudaSuccess;
-#define CK_W4A8_ROWSPLIT(NT, CPW)                                                                  \
+#define CK_W4A8_ROWSPLIT_A(NT, CPW, A4)                                                            \
   {                                                                                                \
-    auto kern = w4a8_rowsplit_kernel<NT, CPW>;                                                     \
+    auto kern = w4a8_rowsplit_kernel<NT, CPW, A4>;                                                 \
     struct Tag {};                                                                                 \
     e = set_smem_max<Tag>(kern, total, smax);                                                      \
     if (e == cudaSuccess) e = launch_pdl(kern, dim3(grid), dim3(nthreads), total, st, tw, p);      \
+  }
+#define CK_W4A8_ROWSPLIT(NT, CPW)                                                                  \
+  {                                                                                                \
+    if (a4) CK_W4A8_ROWSPLIT_A(NT, CPW, true)                                                      \
+    else CK_W4A8_ROWSPLIT_A(NT, CPW, false)                                                        \
   }
   if (nt == 1) {
     if (cpw <= 1) CK_W4A8_ROWSPLIT(1, 1)
@@ -1061,6 +1095,7 @@ ck_status gemv_w4a8_rowsplit(const int8_t* xq, const float* x_scale, int64_t M, 
     else CK_W4A8_ROWSPLIT(4, 2)
   }
 #undef CK_W4A8_ROWSPLIT
+#undef CK_W4A8_ROWSPLIT_A
   if (e != cudaSuccess) return fail(CK_ERR_CUDA, "gemv_w4a8: %s", cudaGetErrorString(e));
   return launch_status("gemv_w4a8");
 }

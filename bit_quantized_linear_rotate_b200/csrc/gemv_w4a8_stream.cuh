@@ -98,7 +98,10 @@ __device__ __forceinline__ void cta_rows(int N, int& n0, int& n1) {
 
 // NT: token groups of 8 (M <= 8 NT); CPW: 128-column chunks per consumer warp
 // (K <= NC * 128 * CPW).
-template <int NT, int CPW>
+// A4: the activations are int4 codes packed two per byte (offset binary u = q + 8,
+// low nibble = even column, (M, K / 2) bytes) instead of int8: half the bytes every
+// CTA pulls from L2.
+template <int NT, int CPW, bool A4 = false>
 __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
     w4a8_rowsplit_kernel(const __grid_constant__ CUtensorMap tm_w, const Params p) {
   constexpr int NC = cons_warps(NT), W_PROD = NC;   // then the epilogue warp, NC + 1, if NT == 1
@@ -193,13 +196,21 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
         for (int ci = 0; ci < CPW; ++ci) {
           const int c = warp + NC * ci;
           uint4 a0 = make_uint4(0, 0, 0, 0), a1 = a0;
-          if (c < nchunk && tok < p.M) {
-            const uint4* xp = reinterpret_cast<const uint4*>(p.xq + (int64_t)tok * p.K + c * 128 + 32 * t);
-            a0 = __ldg(xp);
-            a1 = __ldg(xp + 1);
+          if constexpr (A4) {   // word j: the 8 codes of k = 32t + 8j .. + 7; u = 8 (code 0) where absent
+            a0 = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+            if (c < nchunk && tok < p.M)
+              a0 = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.xq) +
+                                                        (int64_t)tok * (p.K >> 1) + c * 64 + 16 * t));
+            bf[ci][0][0][nt] = a0.x; bf[ci][1][0][nt] = a0.y; bf[ci][2][0][nt] = a0.z; bf[ci][3][0][nt] = a0.w;
+          } else {
+            if (c < nchunk && tok < p.M) {
+              const uint4* xp = reinterpret_cast<const uint4*>(p.xq + (int64_t)tok * p.K + c * 128 + 32 * t);
+              a0 = __ldg(xp);
+              a1 = __ldg(xp + 1);
+            }
+            bf[ci][0][0][nt] = a0.x; bf[ci][0][1][nt] = a0.y; bf[ci][1][0][nt] = a0.z; bf[ci][1][1][nt] = a0.w;
+            bf[ci][2][0][nt] = a1.x; bf[ci][2][1][nt] = a1.y; bf[ci][3][0][nt] = a1.z; bf[ci][3][1][nt] = a1.w;
           }
-          bf[ci][0][0][nt] = a0.x; bf[ci][0][1][nt] = a0.y; bf[ci][1][0][nt] = a0.z; bf[ci][1][1][nt] = a0.w;
-          bf[ci][2][0][nt] = a1.x; bf[ci][2][1][nt] = a1.y; bf[ci][3][0][nt] = a1.z; bf[ci][3][1][nt] = a1.w;
         }
       }
 #pragma unroll
@@ -209,10 +220,20 @@ __global__ void __launch_bounds__(threads_for(NT), NT == 1 ? 2 : 1)
         for (int ci = 0; ci < CPW; ++ci)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint32_t w0 = bf[ci][j][0][nt], w1 = bf[ci][j][1][nt];
-            xs_g = __dp4a((int)w0, 0x01010101, __dp4a((int)w1, 0x01010101, xs_g));
-            bf[ci][j][0][nt] = __byte_perm(w0, w1, 0x6420);
-            bf[ci][j][1][nt] = __byte_perm(w0, w1, 0x7531);
+            if constexpr (A4) {
+              // even / odd k nibbles to signed bytes: (u + 0x78) ^ 0x80 = u - 8, no carry between bytes
+              const uint32_t w = bf[ci][j][0][nt];
+              const uint32_t ev = ((w & 0x0F0F0F0Fu) + 0x78787878u) ^ 0x80808080u;
+              const uint32_t od = (((w >> 4) & 0x0F0F0F0Fu) + 0x78787878u) ^ 0x80808080u;
+              xs_g = __dp4a((int)ev, 0x01010101, __dp4a((int)od, 0x01010101, xs_g));
+              bf[ci][j][0][nt] = ev;
+              bf[ci][j][1][nt] = od;
+            } else {
+              const uint32_t w0 = bf[ci][j][0][nt], w1 = bf[ci][j][1][nt];
+              xs_g = __dp4a((int)w0, 0x01010101, __dp4a((int)w1, 0x01010101, xs_g));
+              bf[ci][j][0][nt] = __byte_perm(w0, w1, 0x6420);
+              bf[ci][j][1][nt] = __byte_perm(w0, w1, 0x7531);
+            }
           }
         xs_g += __shfl_xor_sync(0xffffffffu, xs_g, 1);
         xs_g += __shfl_xor_sync(0xffffffffu, xs_g, 2);

@@ -211,8 +211,9 @@ ck_status ck_linear_w4a4(const void* x, ck_dtype xt, int64_t M, int64_t K, int64
  * The two phases of ck_linear_w4a4, callable separately (to time or overlap
  * them). Phase 1 rotates and quantizes x into `workspace`: the int4 codes
  * stored one per byte (as comfy-kitchen PR #212 "Related work" notes, #201
- * does away with the activation pack/unpack) and the row scales, in a layout
- * private to the library that depends only on (M, K). Phase 2 multiplies
+ * does away with the activation pack/unpack) -- for small batches packed two
+ * per byte, since every SM of that route reads all of them -- and the row
+ * scales, in a layout private to the library that depends only on (M, K). Phase 2 multiplies
  * those codes with the packed int4 weights and applies the rowwise-scale
  * epilogue: on the tensor-core GEMM, or for small batches (M <= 64, K <= 4096,
  * K % 128 == 0) on the streaming decode-GEMV kernels, which keep every SM

@@ -357,12 +357,22 @@ def _small_m_route(M, K):
     return M <= 64 and K % 128 == 0 and K <= 4096
 
 
-def _linear_workspace(ws, M, K):
-    """(codes in natural column order, scales, row sums or None) from the linear's workspace."""
-    nq = _a256(M * K)
-    q = ws[:M * K].view(torch.int8).view(M, K).cpu().numpy().astype(np.int64)
+def _linear_workspace(ws, M, K, bits=4):
+    """(codes in natural column order, scales, row sums or None) from the linear's workspace.
+
+    Small batches keep int4 codes packed two per byte (offset binary, low nibble = even column)
+    followed by room for them one per byte; int8 codes (the W4A8 linear) one per byte."""
+    small = _small_m_route(M, K)
+    nq = _a256(M * K // 2) + _a256(M * K) if small else _a256(M * K)
     s = ws[nq:nq + 4 * M].view(torch.float32).cpu().numpy()
-    if _small_m_route(M, K):
+    if small and bits == 4:
+        b = ws[:M * K // 2].cpu().numpy().reshape(M, K // 2).astype(np.int64)
+        q = np.empty((M, K), dtype=np.int64)
+        q[:, 0::2] = (b & 15) - 8
+        q[:, 1::2] = (b >> 4) - 8
+        return q, s, None
+    q = ws[:M * K].view(torch.int8).view(M, K).cpu().numpy().astype(np.int64)
+    if small:
         return q, s, None
     perm = np.array([0, 2, 4, 6, 1, 3, 5, 7])
     nat = np.empty_like(q)
@@ -407,7 +417,7 @@ def _linear_full_config(ck, w, chunk_rows=2048, bits=4):
     torch.cuda.synchronize()
     # the quantized activations the GEMM consumed (workspace: int8 codes with each 8-column group
     # stored as columns (0 2 4 6 1 3 5 7), row scales, row sums of the codes)
-    qa_all, sa_all, rs_all = _linear_workspace(ws, w.M, w.K)
+    qa_all, sa_all, rs_all = _linear_workspace(ws, w.M, w.K, bits)
     qmax = O.QMAX[bits]
     assert qa_all.min() >= -qmax and qa_all.max() <= qmax
     if rs_all is not None:
@@ -486,7 +496,7 @@ def test_linear_w4a8_equals_rotate_quant_plus_gemm_w4a8(ck, M, K, N):
     q8, s8 = ck.rotate_quant_rowwise(x, 64, 8)
     y0 = ck.gemm_w4a8(q8, s8, wp, sw, bias=b)
     assert torch.equal(y1, y0)
-    q, s, rs = _linear_workspace(ws, M, K)
+    q, s, rs = _linear_workspace(ws, M, K, bits=8)
     np.testing.assert_array_equal(q, q8.cpu().numpy().astype(np.int64))
     np.testing.assert_array_equal(s, s8.cpu().numpy())
     if rs is not None:
