@@ -13,10 +13,10 @@
 // * Work split. CTA b of a grid of G (one per SM) owns output rows
 //   [n0, n1), whole octets of rows split evenly, moved in 16-row tiles (the
 //   m16 operand of mma.sync.m16n8k32 u8 x s8; the tokens, in NT groups of 8,
-//   are the n8 operands). A last tile that would run
-//   past n1 is moved back to end at n1 (its first rows, already produced by
-//   the previous tile, are computed again and not stored), so no CTA carries
-//   more than one tile beyond the average.
+//   are the n8 operands). A last tile that would run past n1 is moved back to
+//   end at n1 (its first rows, already produced by the previous tile, are
+//   computed again and not stored), so no CTA carries more than one tile
+//   beyond the average.
 // * Weight tiles. One tensor copy per tile through a 3-D view of the weight
 //   matrix ([K/128 slices][rows][64 B], 64-byte swizzle, see wtile_addr).
 //   The producer warp reads only constant data, so it does not wait for the
@@ -32,15 +32,20 @@
 //   queue ahead of this call's activation loads (measured: 6.8 -> 6.3 us a
 //   call at M = 1..4, K = 4096, N = 12288).
 // * Compute. NC consumer warps split K (8 for one token group, 16 and one CTA
-//   per SM for more); each holds its activation fragments in registers. A packed word costs two logical ops: the low nibbles (even k)
-//   and the high nibbles left in place (16 x odd-k value) go to two MMAs with
-//   separate accumulators, and the high sum, a multiple of 16, is shifted
-//   back exactly. Nibbles enter unsigned: sum (u - 8) x = sum u x - 8 sum x.
+//   per SM for more); each holds its activation fragments in registers (read
+//   as int8, or as int4 codes packed two per byte for the small-batch linear,
+//   A4). A packed weight word costs two logical ops: the low nibbles (even k)
+//   and the high nibbles (odd k) go to two MMAs; with one token group the
+//   high nibbles stay in place (16 x the value) in an accumulator of their
+//   own, shifted back exactly at the end, with more groups they are shifted
+//   down first. Nibbles enter unsigned: sum (u - 8) x = sum u x - 8 sum x.
 // * Reduction. Each consumer warp adds its partial tile into a shared-memory
 //   slot of that tile (integer adds commute: the result does not depend on
-//   the order) and arrives on the tile's barrier; an epilogue warp waits for
-//   the tiles in order and writes y. No warp waits for the epilogue, and no
-//   memory fence sits on the consumers' path.
+//   the order). One token group: the warp arrives on the tile's barrier and
+//   an epilogue warp waits for the tiles in order and writes y; no warp waits
+//   for the epilogue, and no memory fence sits on the consumers' path. More
+//   groups: the consumer warps meet at a named barrier and write the tile's
+//   outputs themselves, one per lane.
 // All barrier waits are bounded; a timeout sets the device error word.
 #pragma once
 
@@ -64,7 +69,7 @@ __host__ __device__ constexpr int cons_warps(int nt) { return nt == 1 ? 8 : 16; 
 __host__ __device__ constexpr int threads_for(int nt) { return (cons_warps(nt) + (nt == 1 ? 2 : 1)) * 32; }
 
 struct Params {
-  const int8_t* xq;               // (M, K)
+  const int8_t* xq;               // (M, K) int8, or (M, K / 2) packed int4 codes (A4)
   const float* xs;                // (M)
   const __nv_bfloat16* sw;        // (N)
   const __nv_bfloat16* bias;      // (N) or null
