@@ -72,6 +72,11 @@ def test_workspace_bytes(ck):
     assert ck.linear_w4a4_workspace_bytes(8192, 3840) == 8192 * 3840 + 8192 * 4 + 8192 * 4
     assert ck.linear_w4a4_workspace_bytes(3, 64) == 256 + 256 + 12
     assert ck.linear_w4a4_workspace_bytes(0, 64) == 0
+    # small batches (M <= 64, K % 128 == 0, K <= 4096): the codes packed two per byte, then
+    # room for them one per byte
+    assert ck.linear_w4a4_workspace_bytes(32, 3840) == 32 * 1920 + 32 * 3840 + 256 + 32 * 4
+    assert ck.linear_w4a4_workspace_bytes(3, 128) == 256 + 512 + 256 + 12
+    assert ck.linear_w4a8_workspace_bytes(32, 3840) == ck.linear_w4a4_workspace_bytes(32, 3840)
 
 
 def _rq(ck, **kw):
