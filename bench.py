@@ -493,9 +493,13 @@ def time_other_configs(ck, dev, peaks):
             ws = torch.empty(ck.linear_w4a4_workspace_bytes(M, K), device=dev, dtype=torch.uint8)
             ms = time_rotating(lambda c: ck.linear_w4a4_quantize(xs[c], G, ws), R, 100, 5)
             nbytes = M * K * 2 + M * K + 8 * M
+            # the same time on the survey's algorithmic bytes of a1-a3: x, the packed int4 codes
+            # and the row scales (the phase stores its codes one per byte plus row sums instead)
+            alg = M * K * 2 + M * K // 2 + 4 * M
             out[f"linear_quantize_M{M}_K{K}_G{G}"] = {
                 "us": round(ms * 1e3, 2), "GBps": round(nbytes / (ms * 1e-3) / 1e9, 1),
-                "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "copies": R}
+                "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "frac_hbm_packed_codes_bytes": round(alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "copies": R}
         del xs
     return out
 
