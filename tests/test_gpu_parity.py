@@ -273,6 +273,7 @@ def test_gemm_w4a8_and_s8_epilogue_bit_exact(ck, M, K, N):
     (129, 768, 260, 256, False, torch.float16),
     (300, 256, 520, 16, True, torch.bfloat16),
     (64, 3840, 3840, 64, False, torch.bfloat16),
+    (24, 1024, 264, 16, True, torch.float16),      # small-batch route, fp16, packed codes
 ])
 def test_linear_w4a4_matches_oracle(ck, M, K, N, G, bias, dtype):
     d = WL.small_linear_inputs(M, K, N, seed=M + K, n_outlier_cols=K // 100, dtype=dtype, with_bias=bias)
